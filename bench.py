@@ -1,0 +1,458 @@
+#!/usr/bin/env python
+"""Benchmark of the gated-delta-rule QDQ-state hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One JSON line on stdout (rank 0).  The headline `value` is GDN prefill
+tokens/s on the GDN-prefill workload (B=4, H=16, T=4096, d_k=d_v=128, bf16
+q/k/v, fp32 gates/state, FP8 E4M3 tile-64 state QDQ at every 64-token
+chunk): one step = one gdn_prefill call over the whole batch with inputs
+resident in HBM.  The serving-decode workload (256 sequences x 32 heads,
+d=128, INT8 g32 state QDQ after every token, 512 single-token gdn_decode
+calls) is measured in the same run and reported under "decode".
+
+With N > 1 (torchrun, one rank per GPU) every rank runs its own copy of the
+workload (independent sequences; no collective on the data path), the step
+time is the max over ranks, and `value` counts the tokens of all ranks.
+
+`--impl reference` times the CPU oracle (fp64 token recurrence + fp32
+codecs) on a bounded sample of the same workload on the host cores.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "GDN prefill tokens/s + QDQ-state decode updates/s; % of TC / HBM roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "source": "fallback"}
+
+
+def load_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        d["source"] = "measured"
+        return d
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS)
+
+
+# ------------------------------------------------------------ workload math
+def prefill_bytes(B, T, H, dk, dv, in_bytes, state_in: bool, per_key: bool) -> int:
+    """Algorithmic HBM bytes of one prefill call: q, k, v read, o written
+    (in dtype), g and beta read (fp32), state written (and read if given)."""
+    tok = B * T * H
+    b = tok * (2 * dk + dv) * in_bytes + tok * dv * in_bytes
+    b += tok * 4 * (dk if per_key else 1) + tok * 4
+    b += B * H * dk * dv * 4 * (2 if state_in else 1)
+    return b
+
+
+def prefill_flops(B, T, H, dk, dv, C=64) -> int:
+    """Dense algorithmic flops of the chunked WY form per call: per chunk
+    K K^T, Q K^T and W = T (bK): 3 * 2*C*C*d_k; U = T (bV) and Aqk Vn:
+    2 * 2*C*C*d_v; W H0, Q H0 and K^T Vn: 3 * 2*C*d_k*d_v."""
+    per_chunk = 3 * 2 * C * C * dk + 2 * 2 * C * C * dv + 3 * 2 * C * dk * dv
+    return B * H * (T // C) * per_chunk + (B * H * (T % C) * per_chunk) // C
+
+
+def decode_bytes_per_update(dk, dv, in_bytes, per_key: bool) -> int:
+    """State read + write (fp32), q, k, v read and o written, g and beta."""
+    return 2 * 4 * dk * dv + (2 * dk + dv) * in_bytes + dv * in_bytes + 4 * (dk if per_key else 1) + 4
+
+
+# ------------------------------------------------------------ clock sampler
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples, tagged with host time."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int, period_ms: int = 50):
+        self.samples = []
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 f"-lms={period_ms}", f"-i={gpu_index}"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.samples.append((time.time(), parts))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0: float, t1: float) -> dict:
+        inside = [p for (t, p) in self.samples if t0 <= t <= t1]
+        window = "timed region"
+        if not inside:  # region shorter than the sampling period: nearest samples
+            inside = [p for (t, p) in self.samples if t0 - 0.5 <= t <= t1 + 0.5]
+            window = "timed region +-0.5 s"
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(p[1]) for p in inside if num(p[1]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for p in inside for i in range(4) if p[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": num(inside[0][2]), "reasons": reasons,
+                "power_w_max": max((num(p[3]) or 0.0) for p in inside),
+                "samples": len(inside), "window": window}
+
+
+# ------------------------------------------------------------ distributed
+class Dist:
+    def __init__(self, n_gpus: int):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+        if self.world != n_gpus:
+            raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={self.world}")
+
+    def init(self, backend: str):
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg:
+            self.pg.barrier()
+
+    def max(self, x: float) -> float:
+        if not self.pg:
+            return x
+        import torch
+        dev = "cuda" if self.pg.get_backend() == "nccl" else "cpu"
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+# ------------------------------------------------------------ our arm
+def cpu_baseline_prefill(case, inp, max_seconds: float = 12.0) -> dict:
+    """The oracle as it stands, on whole sequences of the workload (all
+    heads), on this host's cores; tokens/s scaled from the sample."""
+    import oracle
+    threads = len(os.sched_getaffinity(0))
+    T = case.T
+    done, t_total = 0, 0.0
+    for s in range(case.n_seq):
+        sl = slice(s, s + 1)
+        t0 = time.perf_counter()
+        oracle.recurrence(inp["q"][sl], inp["k"][sl], inp["v"][sl], inp["g"][sl],
+                          inp["beta"][sl], None, oracle.dense_cu_seqlens(1, T),
+                          per_key_gate=case.gate == "per_key", qdq=case.qdq, n_threads=threads)
+        t_total += time.perf_counter() - t0
+        done += 1
+        if t_total * (done + 1) / done > max_seconds:
+            break
+    return {"value": done * T / t_total, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{done} of {case.n_seq} sequences ({T} tokens x {case.H} heads each), "
+                      f"fp64 token recurrence + fp32 {case.qdq} codec, OpenMP over heads",
+            "seconds": round(t_total, 3)}
+
+
+def cpu_baseline_decode(case, inp, state) -> dict:
+    import oracle
+    threads = len(os.sched_getaffinity(0))
+    n_seq = 64
+    sl = (slice(0, 1), slice(0, n_seq))
+    t0 = time.perf_counter()
+    oracle.decode(inp["dec_q"][sl], inp["dec_k"][sl], inp["dec_v"][sl], inp["dec_g"][sl],
+                  inp["dec_beta"][sl], state[:n_seq], per_key_gate=False, qdq=case.qdq,
+                  n_threads=threads)
+    dt = time.perf_counter() - t0
+    return {"value": n_seq * case.H / dt, "unit": "updates/s", "cores": threads, "kind": "oracle",
+            "sample": f"1 token of {n_seq} of {case.n_seq} sequences x {case.H} heads",
+            "seconds": round(dt, 3)}
+
+
+def run_ours(args, dist: Dist) -> dict:
+    import torch
+
+    import gdn_synth as gs
+    import state_quantized_recurrence_b200 as sqr
+
+    peaks = load_peaks()
+    torch.cuda.set_device(dist.local)
+    dist.init("nccl")
+    dev = torch.device("cuda", dist.local)
+    stream = torch.cuda.current_stream(dev)
+    sampler = ClockSampler(dist.local)
+
+    # ---------------- prefill (headline) ----------------
+    case = gs.CONFIGS["gdn_prefill"]
+    if args.small:
+        case = gs.small_case("gdn_prefill", n_seq=1, H=16, T=1024)
+    inp = gs.generate(case)
+    d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    o = torch.empty(d["v"].shape, dtype=d["q"].dtype, device=dev)
+    st = torch.empty((case.n_seq, case.H, case.d_k, case.d_v), dtype=torch.float32, device=dev)
+
+    def step():
+        sqr.gdn_prefill_into(d["q"], d["k"], d["v"], d["g"], d["beta"], None, None, o, st,
+                             qdq=case.qdq)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    sqr.check_last_error(where="prefill warm-up")
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    t_wall0 = time.time()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    t_wall1 = time.time()
+    dist.barrier()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    ms_max = dist.max(ms)
+    clocks = sampler.summary(t_wall0, t_wall1)
+
+    B, T, H, dk, dv = case.n_seq, case.T, case.H, case.d_k, case.d_v
+    tokens = B * T
+    value = dist.world * tokens / (ms_max / 1e3)
+    nbytes = prefill_bytes(B, T, H, dk, dv, 2, False, case.gate == "per_key")
+    flops = prefill_flops(B, T, H, dk, dv)
+    gbs = nbytes / (ms / 1e3) / 1e9
+    tfs = flops / (ms / 1e3) / 1e12
+    roofline = {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": None,
+                "kernel": "prefill (one launch per step)", "bytes_per_launch": nbytes,
+                "peak_source": peaks["source"],
+                "tensor": {"achieved": round(tfs, 2), "peak": peaks["bf16_tflops"],
+                           "unit": "TFLOP/s", "frac": round(tfs / peaks["bf16_tflops"], 4),
+                           "flops_per_launch": flops}}
+
+    # e2e through the C ABI from pinned host buffers (copies inside the timed region)
+    host = {k: d[k].cpu().pin_memory() for k in ("q", "k", "v", "g", "beta")}
+    o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    st_h = torch.empty(st.shape, dtype=st.dtype).pin_memory()
+    e2e_steps = max(3, min(args.steps, 10))
+
+    def e2e_step():
+        for k in host:
+            d[k].copy_(host[k], non_blocking=True)
+        step()
+        o_h.copy_(o, non_blocking=True)
+        st_h.copy_(st, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    ev0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    ms_e2e = dist.max(ev0.elapsed_time(ev1) / e2e_steps)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = o_h.numel() * o_h.element_size() + st_h.numel() * st_h.element_size()
+    e2e = {"value": dist.world * tokens / (ms_e2e / 1e3), "unit": "tokens/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_e2e, 4),
+           "steps": e2e_steps}
+
+    cpu = None
+    if dist.world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline_prefill(case, inp)
+    del d, host, o, st, o_h, st_h
+    torch.cuda.empty_cache()
+
+    # ---------------- decode ----------------
+    dec = None
+    if not args.no_decode:
+        dec = run_decode(args, dist, dev, stream, sampler, peaks)
+
+    sampler.stop()
+    res = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": dist.world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_max, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": f"gdn_prefill B={B} H={H} T={T} d_k={dk} d_v={dv}, bf16 q/k/v, "
+                               f"fp32 g/beta/state, {case.qdq} state QDQ, zero initial state",
+                   "global_batch": B * dist.world, "seq_len": T,
+                   "l2": f"inputs {nbytes / 1e6:.0f} MB > 126 MB L2, no flush",
+                   "parallelism": f"dp{dist.world} (independent sequences per rank)"},
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps,
+        "clocks": clocks, "decode": dec, "impl": "ours",
+    }
+    dist.close()
+    return res
+
+
+def run_decode(args, dist, dev, stream, sampler, peaks) -> dict:
+    import torch
+
+    import gdn_synth as gs
+    import state_quantized_recurrence_b200 as sqr
+
+    case = gs.CONFIGS["serving_decode"]
+    if args.small:
+        case = gs.small_case("serving_decode", n_seq=64, decode_steps=16)
+    inp = gs.generate(case)
+    S_steps = case.decode_steps
+    dq, dk_, dv_ = inp["dec_q"].to(dev), inp["dec_k"].to(dev), inp["dec_v"].to(dev)
+    dg, db = inp["dec_g"].to(dev), inp["dec_beta"].to(dev)
+    state0 = inp["state_in"].to(dev)
+    state = state0.clone()
+    o = torch.empty((S_steps,) + tuple(dv_.shape[1:]), dtype=dq.dtype, device=dev)
+
+    def run_all():
+        for t in range(S_steps):
+            sqr.gdn_decode_into(dq[t], dk_[t], dv_[t], dg[t], db[t], state, o[t], qdq=case.qdq)
+
+    # warm-up, then capture the whole token loop in one CUDA graph
+    for _ in range(max(1, args.warmup)):
+        state.copy_(state0)
+        run_all()
+    torch.cuda.synchronize(dev)
+    sqr.check_last_error(where="decode warm-up")
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        run_all()
+    state.copy_(state0)
+    graph.replay()
+    torch.cuda.synchronize(dev)
+    reps = 3
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    t_wall0 = time.time()
+    ev0.record(stream)
+    for _ in range(reps):
+        graph.replay()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    t_wall1 = time.time()
+    dist.barrier()
+    ms_loop = dist.max(ev0.elapsed_time(ev1) / reps)
+    updates = case.n_seq * case.H * S_steps
+    ups = dist.world * updates / (ms_loop / 1e3)
+    bpu = decode_bytes_per_update(case.d_k, case.d_v, 2, False)
+    ms_tok = ms_loop / S_steps
+    gbs = case.n_seq * case.H * bpu / (ms_tok / 1e3) / 1e9
+    cpu = None
+    if dist.world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline_decode(case, inp, inp["state_in"])
+    del graph
+    return {"metric": "QDQ-state decode updates/s", "value": round(ups, 1), "unit": "updates/s",
+            "sequence_tokens_per_s": round(ups / case.H, 1),
+            "workload": f"serving_decode {case.n_seq} seq x H={case.H}, d=128, bf16, "
+                        f"{case.qdq}, {S_steps} single-token calls in one CUDA graph",
+            "ms_per_token_step": round(ms_tok, 5), "reps": reps,
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
+                         "traffic": None, "bytes_per_update": bpu,
+                         "peak_source": peaks["source"]},
+            "gpu_launches": S_steps * reps, "clocks": sampler.summary(t_wall0, t_wall1),
+            "cpu_baseline": cpu}
+
+
+# ------------------------------------------------------------ reference arm
+def run_reference(args, dist: Dist) -> dict | None:
+    """The oracle, as it stands, on the host cores: each step is a bounded
+    sample (one sequence, all heads, the first 1024 tokens) of the workload."""
+    if dist.rank != 0:
+        return None
+    import gdn_synth as gs
+    import oracle
+
+    case = gs.CONFIGS["gdn_prefill"]
+    inp = gs.generate(case)
+    threads = len(os.sched_getaffinity(0))
+    Ts = 4096
+    sl = (slice(0, 1), slice(0, Ts))
+
+    def step():
+        oracle.recurrence(inp["q"][sl], inp["k"][sl], inp["v"][sl], inp["g"][sl],
+                          inp["beta"][sl], None, oracle.dense_cu_seqlens(1, Ts),
+                          per_key_gate=False, qdq=case.qdq, n_threads=threads)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    value = Ts / dt
+    sample = f"1 sequence x {case.H} heads x {Ts} tokens of the gdn_prefill workload per step"
+    return {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": dist.world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": f"gdn_prefill B={case.n_seq} H={case.H} T={case.T} d=128, "
+                                   f"{case.qdq} (sampled)", "global_batch": case.n_seq,
+                       "seq_len": case.T, "parallelism": "host cores"},
+            "impl": "reference",
+            "cpu_baseline": {"value": round(value, 1), "unit": "tokens/s", "cores": threads,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 1), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--small", action="store_true", help="small case (profiling captures)")
+    args = ap.parse_args()
+    if args.warmup < 3 and not args.small:
+        raise SystemExit("--warmup must be >= 3")
+    dist = Dist(args.gpus)
+    if args.impl == "reference":
+        res = run_reference(args, dist)
+    else:
+        res = run_ours(args, dist)
+    if res is not None and dist.rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

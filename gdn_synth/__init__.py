@@ -13,7 +13,8 @@ drawn per key channel.  Random initial states are N(0, 0.05^2) in fp32.
 
 Draw order for one case, all from one ``torch.Generator('cpu')`` seeded with
 ``case.seed``: lengths (packed cases only), q, k, v, beta-logit, gate-logit,
-initial state, then per decode step q, k, v, beta-logit, gate-logit.  Every
+initial state, then the decode tokens' q, k, v, beta-logit and gate-logit,
+each drawn for all decode steps at once ([steps, n_seq, H, ...]).  Every
 draw is fp32 on the CPU; q/k/v are cast to the case's dtype at the end.
 """
 
@@ -148,17 +149,10 @@ def generate(case: Case) -> dict:
 
     if case.decode_steps > 0:
         S, N = case.decode_steps, case.n_seq
-        dq = torch.empty((S, N, H, dk), dtype=dt)
-        dkk = torch.empty((S, N, H, dk), dtype=dt)
-        dvv = torch.empty((S, N, H, dv), dtype=dt)
-        dbeta = torch.empty((S, N, H), dtype=torch.float32)
-        gs = (N, H, dk) if case.gate == "per_key" else (N, H)
-        dg = torch.empty((S,) + gs, dtype=torch.float32)
-        for s in range(S):
-            dq[s] = _unit_normal_rows(gen, (N, H, dk)).to(dt)
-            dkk[s] = _unit_normal_rows(gen, (N, H, dk)).to(dt)
-            dvv[s] = torch.randn((N, H, dv), generator=gen, dtype=torch.float32).to(dt)
-            dbeta[s] = _beta(gen, (N, H))
-            dg[s] = _log_gate(gen, gs)
-        out.update(dec_q=dq, dec_k=dkk, dec_v=dvv, dec_beta=dbeta, dec_g=dg)
+        gs = (S, N, H, dk) if case.gate == "per_key" else (S, N, H)
+        out["dec_q"] = _unit_normal_rows(gen, (S, N, H, dk)).to(dt)
+        out["dec_k"] = _unit_normal_rows(gen, (S, N, H, dk)).to(dt)
+        out["dec_v"] = torch.randn((S, N, H, dv), generator=gen, dtype=torch.float32).to(dt)
+        out["dec_beta"] = _beta(gen, (S, N, H))
+        out["dec_g"] = _log_gate(gen, gs)
     return out

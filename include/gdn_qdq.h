@@ -1,0 +1,142 @@
+/*
+ * gdn_qdq.h - C ABI of the B200 (sm_100a) gated-delta-rule library with a
+ * fake-quantized (QDQ) recurrent state.
+ *
+ * The operations follow the GatedDeltaNet / KDA state-QAT pages (the
+ * "linear_attention" QAT series of NVIDIA Model-Optimizer):
+ *   - prefix ("chunked prefix", PR #2519 What section; "64-token chunks" and
+ *     the "WY-transformed W", PR #2497 What section): the sequence is cut into
+ *     64-token chunks, each chunk is solved in the WY form with an exact
+ *     triangular solve (PR #2507 What section: "exact triangular solve
+ *     remains the default"), and the state is carried chunk to chunk;
+ *   - suffix ("recurrent suffix", recurrent_decode, PR #2519 What section):
+ *       S_t = S_{t-1} diag(alpha_t);  u_t = beta_t (v_t - S_t k_t);
+ *       S_t += u_t k_t^T;  o_t = S_t q_t / sqrt(d_k);
+ *   - state QDQ at every 64-token chunk boundary of the prefix and after every
+ *     decode token: dynamic FP8 E4M3 with one scale per (all d_k keys x 64
+ *     value columns) tile per sequence and head, scale = amax / 448 with a
+ *     zero guard (PR #2497 What section); or dynamic INT8 with groups of 32
+ *     along the last axis, scale = amax / 127, round half to even, clamp to
+ *     [-127, 127] (PR #2519 commit notes, recipe
+ *     linear_attention_state_int8_block32_dynamic);
+ *   - fp32 working values for the state and the gates, bf16 or fp32 q/k/v
+ *     promoted to fp32 (PR #2519 commit notes).
+ *
+ * Layouts (all row-major, contiguous):
+ *   state  fp32 [n_seq, H, d_k, d_v]: the transpose H = S^T of the pages'
+ *          state, row = key, column = value, so the FP8 tile is d_k rows x
+ *          64 columns and INT8 groups run along d_v (the last axis).
+ *   q, k   [.., H, d_k]; v, o [.., H, d_v] in the dtype `dt`;
+ *   g      fp32 natural-log gates (alpha = exp(g) in (0, 1]): [.., H] for
+ *          GDN (GDN_GATE_SCALAR) or [.., H, d_k] for KDA (GDN_GATE_PER_KEY);
+ *   beta   fp32 [.., H].
+ *
+ * Ownership: every pointer is caller-owned memory; the library allocates
+ * nothing and keeps no reference after a call returns.  Pointers are device
+ * pointers unless a function says otherwise.
+ *
+ * Asynchrony and errors: argument errors are detected on the host and
+ * returned before anything is launched (nothing is written).  Compute calls
+ * are asynchronous on `cuda_stream` (a cudaStream_t; NULL = the legacy
+ * default stream).  Errors found on the device (a malformed cu_seqlens, a
+ * bounded wait that ran out) are recorded in a per-device error word that
+ * gdn_last_error() reports.  There is no fallback of any kind: an
+ * unsupported combination returns GDN_ERR_UNSUPPORTED.
+ *
+ * Supported: d_k, d_v in {64, 128}; dt in {bf16, f32}; q, k, v, o and the
+ * states 16-byte aligned, g and beta 4-byte aligned.
+ */
+#ifndef GDN_QDQ_H_
+#define GDN_QDQ_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = 1,  /* bad pointer, size, alignment or cu_seqlens */
+    GDN_ERR_UNSUPPORTED = 2,  /* valid but unsupported combination */
+    GDN_ERR_CUDA = 3,         /* a CUDA runtime call failed */
+    GDN_ERR_TIMEOUT = 4       /* a bounded device-side wait ran out */
+} gdn_status;
+
+typedef enum {
+    GDN_QDQ_NONE = 0,
+    GDN_QDQ_FP8_E4M3_TILE64 = 1, /* one scale per (d_k x 64 value columns) */
+    GDN_QDQ_INT8_GROUP32 = 2,    /* groups of 32 along d_v */
+    GDN_QDQ_INT8_GROUP16 = 3,    /* groups of 16 along d_v */
+    GDN_QDQ_INT8_GROUP64 = 4     /* groups of 64 along d_v */
+} gdn_qdq_mode;
+
+typedef enum { GDN_DTYPE_BF16 = 0, GDN_DTYPE_F32 = 1 } gdn_dtype;
+
+typedef enum {
+    GDN_GATE_SCALAR = 0,   /* GDN: one log-gate per token and head */
+    GDN_GATE_PER_KEY = 1   /* KDA: one log-gate per token, head, key channel */
+} gdn_gate_kind;
+
+/*
+ * gdn_prefill - chunked prefix over n_seq sequences.
+ *
+ * Dense layout (cu_seqlens == NULL): q, k, v, o are [n_seq, T, H, d], g is
+ * [n_seq, T, H(, d_k)], beta [n_seq, T, H]; every sequence has T tokens.
+ * Packed layout (cu_seqlens != NULL, int32 device array [n_seq + 1]): the
+ * tensors are [1, T, H, d] with T the total token count; sequence s owns
+ * tokens [cu_seqlens[s], cu_seqlens[s+1]).  cu_seqlens must start at 0, be
+ * non-decreasing and end at T; a violation found on the device skips that
+ * sequence and is reported by gdn_last_error() as GDN_ERR_INVALID_ARG.
+ *
+ * state_in: fp32 [n_seq, H, d_k, d_v] initial states, or NULL for zeros; it
+ *   is used as given (not quantized).  state_out: same shape, receives the
+ *   state after each sequence's last token (QDQ'd unless qdq is NONE or the
+ *   sequence is empty); it may alias state_in exactly (in-place update).
+ * o: [.., H, d_v] in dtype dt; o_t uses the state before that token's QDQ.
+ * The state QDQ runs after tokens 64, 128, ... of each sequence (counted from
+ * its own start) and after its last token.
+ *
+ * Returns GDN_OK after a successful launch (or when there is no work).
+ */
+gdn_status gdn_prefill(const void *q, const void *k, const void *v,
+                       const float *g, const float *beta,
+                       const float *state_in, const int32_t *cu_seqlens,
+                       int n_seq, int T, int H, int d_k, int d_v,
+                       gdn_dtype dt, gdn_gate_kind gk, gdn_qdq_mode qdq,
+                       void *o, float *state_out, void *cuda_stream);
+
+/*
+ * gdn_decode - one decode token for each of n_seq sequences.
+ *
+ * q, k: [n_seq, H, d_k]; v, o: [n_seq, H, d_v] in dtype dt; g: fp32
+ * [n_seq, H] or [n_seq, H, d_k]; beta fp32 [n_seq, H]; state_inout: fp32
+ * [n_seq, H, d_k, d_v], advanced by one token and QDQ'd in place.  o is
+ * computed from the state before its QDQ.
+ */
+gdn_status gdn_decode(const void *q, const void *k, const void *v,
+                      const float *g, const float *beta, float *state_inout,
+                      int n_seq, int H, int d_k, int d_v, gdn_dtype dt,
+                      gdn_gate_kind gk, gdn_qdq_mode qdq, void *o,
+                      void *cuda_stream);
+
+/*
+ * gdn_last_error - synchronize cuda_stream, then read and clear the current
+ * device's error word.  Returns GDN_OK if no device-side error was recorded
+ * since the last call, GDN_ERR_INVALID_ARG for a malformed cu_seqlens,
+ * GDN_ERR_TIMEOUT for a bounded wait that ran out, GDN_ERR_CUDA if the
+ * synchronization itself failed.
+ */
+gdn_status gdn_last_error(void *cuda_stream);
+
+/* gdn_status_string - static, human-readable name of a status code. */
+const char *gdn_status_string(gdn_status s);
+
+/* gdn_version - library version as 10000*major + 100*minor + patch. */
+int gdn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_QDQ_H_ */

@@ -1,0 +1,161 @@
+"""ctypes binding of ``libgdn_qdq.so`` (argument marshalling only)."""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_PKG, "libgdn_qdq.so")
+
+GDN_STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED",
+              3: "GDN_ERR_CUDA", 4: "GDN_ERR_TIMEOUT"}
+GDN_QDQ = {"none": 0, "fp8_tile64": 1, "int8_g32": 2, "int8_g16": 3, "int8_g64": 4}
+GDN_DTYPE = {torch.bfloat16: 0, torch.float32: 1}
+GDN_GATE = {"scalar": 0, "per_key": 1}
+
+
+class GdnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = int(status)
+        super().__init__(f"{where}: {GDN_STATUS.get(self.status, self.status)}")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(library_path):
+        raise ImportError(
+            f"CUDA library {library_path} is missing; build it with "
+            "`python -m state_quantized_recurrence_b200.build` (there is no fallback)")
+    L = ctypes.CDLL(library_path)
+    P, I = ctypes.c_void_p, ctypes.c_int
+    L.gdn_prefill.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P, P, P]
+    L.gdn_prefill.restype = I
+    L.gdn_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, P, P]
+    L.gdn_decode.restype = I
+    L.gdn_last_error.argtypes = [P]
+    L.gdn_last_error.restype = I
+    L.gdn_status_string.argtypes = [I]
+    L.gdn_status_string.restype = ctypes.c_char_p
+    L.gdn_version.argtypes = []
+    L.gdn_version.restype = I
+    return L
+
+
+lib = _load()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need(cond: bool, msg: str):
+    if not cond:
+        raise ValueError(msg)
+
+
+def _check_dev(*ts):
+    for t in ts:
+        if t is not None:
+            _need(t.is_cuda and t.is_contiguous(), "tensors must be contiguous CUDA tensors")
+
+
+def gdn_last_error(stream=None) -> int:
+    """Synchronize the stream and return (and clear) the device error status."""
+    return int(lib.gdn_last_error(_stream(stream)))
+
+
+def check_last_error(stream=None, where: str = "gdn") -> None:
+    s = gdn_last_error(stream)
+    if s != 0:
+        raise GdnError(s, where)
+
+
+def _gate_kind(g: torch.Tensor, lead: int) -> str:
+    return "per_key" if g.dim() == lead + 1 else "scalar"
+
+
+def gdn_prefill_into(q, k, v, g, beta, state_in, cu_seqlens, o, state_out,
+                     qdq: str = "fp8_tile64", stream=None) -> None:
+    """Chunked prefix writing into preallocated ``o`` and ``state_out``.
+
+    Dense: q, k [B, T, H, d_k], v/o [B, T, H, d_v]; packed (cu_seqlens int32
+    [n_seq + 1]): [1, T_total, H, d].  g: fp32 [.., H] or [.., H, d_k];
+    beta fp32 [.., H]; states fp32 [n_seq, H, d_k, d_v].
+    """
+    _check_dev(q, k, v, g, beta, state_in, cu_seqlens, o, state_out)
+    _need(q.dim() == 4 and k.shape == q.shape and v.dim() == 4, "q, k, v must be [B, T, H, d]")
+    B, T, H, d_k = q.shape
+    d_v = v.shape[-1]
+    _need(v.shape[:3] == q.shape[:3] and o.shape == v.shape, "v/o shapes do not match q")
+    _need(q.dtype in GDN_DTYPE and k.dtype == q.dtype and v.dtype == q.dtype and o.dtype == q.dtype,
+          "q, k, v, o must share dtype bf16 or fp32")
+    _need(g.dtype == torch.float32 and beta.dtype == torch.float32, "g and beta must be fp32")
+    _need(beta.shape == q.shape[:3], "beta must be [B, T, H]")
+    gk = _gate_kind(g, 3)
+    _need(g.shape == (q.shape[:3] if gk == "scalar" else q.shape), "g must be [B,T,H] or [B,T,H,d_k]")
+    if cu_seqlens is not None:
+        _need(B == 1 and cu_seqlens.dtype == torch.int32 and cu_seqlens.dim() == 1,
+              "packed layout needs B == 1 and int32 cu_seqlens")
+        n_seq, T_arg = cu_seqlens.numel() - 1, T
+    else:
+        n_seq, T_arg = B, T
+    _need(state_out.shape == (n_seq, H, d_k, d_v) and state_out.dtype == torch.float32,
+          "state_out must be fp32 [n_seq, H, d_k, d_v]")
+    if state_in is not None:
+        _need(state_in.shape == state_out.shape and state_in.dtype == torch.float32,
+              "state_in must be fp32 [n_seq, H, d_k, d_v]")
+    s = lib.gdn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_in),
+                        _ptr(cu_seqlens), n_seq, T_arg, H, d_k, d_v, GDN_DTYPE[q.dtype],
+                        GDN_GATE[gk], GDN_QDQ[qdq], _ptr(o), _ptr(state_out), _stream(stream))
+    if s != 0:
+        raise GdnError(s, "gdn_prefill")
+
+
+def gdn_prefill(q, k, v, g, beta, state_in=None, cu_seqlens=None, qdq: str = "fp8_tile64",
+                stream=None):
+    """Chunked prefix; returns ``(o, state_out)`` (allocated with torch)."""
+    n_seq = q.shape[0] if cu_seqlens is None else cu_seqlens.numel() - 1
+    o = torch.empty(v.shape, dtype=q.dtype, device=q.device)
+    state_out = torch.empty((n_seq, q.shape[2], q.shape[3], v.shape[3]), dtype=torch.float32,
+                            device=q.device)
+    gdn_prefill_into(q, k, v, g, beta, state_in, cu_seqlens, o, state_out, qdq, stream)
+    return o, state_out
+
+
+def gdn_decode_into(q, k, v, g, beta, state, o, qdq: str = "int8_g32", stream=None) -> None:
+    """One decode token per sequence: q, k [N, H, d_k], v/o [N, H, d_v],
+    g [N, H] or [N, H, d_k], beta [N, H]; ``state`` [N, H, d_k, d_v] fp32 is
+    advanced and QDQ'd in place."""
+    _check_dev(q, k, v, g, beta, state, o)
+    _need(q.dim() == 3 and k.shape == q.shape and v.dim() == 3 and o.shape == v.shape,
+          "q, k [N, H, d_k]; v, o [N, H, d_v]")
+    N, H, d_k = q.shape
+    d_v = v.shape[-1]
+    _need(q.dtype in GDN_DTYPE and k.dtype == q.dtype and v.dtype == q.dtype and o.dtype == q.dtype,
+          "q, k, v, o must share dtype bf16 or fp32")
+    _need(g.dtype == torch.float32 and beta.dtype == torch.float32 and beta.shape == (N, H),
+          "g, beta must be fp32; beta [N, H]")
+    gk = _gate_kind(g, 2)
+    _need(g.shape == ((N, H) if gk == "scalar" else (N, H, d_k)), "g must be [N,H] or [N,H,d_k]")
+    _need(state.shape == (N, H, d_k, d_v) and state.dtype == torch.float32,
+          "state must be fp32 [N, H, d_k, d_v]")
+    s = lib.gdn_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state), N, H, d_k,
+                       d_v, GDN_DTYPE[q.dtype], GDN_GATE[gk], GDN_QDQ[qdq], _ptr(o),
+                       _stream(stream))
+    if s != 0:
+        raise GdnError(s, "gdn_decode")
+
+
+def gdn_decode(q, k, v, g, beta, state, qdq: str = "int8_g32", stream=None):
+    o = torch.empty(v.shape, dtype=q.dtype, device=q.device)
+    gdn_decode_into(q, k, v, g, beta, state, o, qdq, stream)
+    return o

@@ -1,0 +1,96 @@
+// Device helpers shared by the decode and prefill kernels: input loads, the
+// state QDQ codecs, and the per-device error word.
+//
+// Codecs (GatedDeltaNet / KDA state-QAT pages): FP8 E4M3 with scale =
+// amax / 448 and a zero guard (PR #2497 What section); INT8 with scale =
+// amax / 127, round half to even and clamp to [-127, 127] (PR #2519 commit
+// notes).  Every step that decides a code is an explicitly rounded IEEE fp32
+// operation (__fdiv_rn, __fmul_rn, rintf, the satfinite E4M3 conversion), so
+// the result does not depend on contraction or approximate division.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gdn {
+
+// Error bits of the device error word.
+constexpr unsigned kErrBadSeqlens = 1u;
+constexpr unsigned kErrTimeout = 2u;
+
+enum QdqKind : int { kQdqNone = 0, kQdqFp8Tile = 1, kQdqInt8 = 2 };
+
+// ---------------------------------------------------------------- loads ----
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+// Four consecutive elements (16-byte aligned for fp32, 8-byte for bf16).
+__device__ __forceinline__ float4 load4(const float *p) {
+  return __ldg(reinterpret_cast<const float4 *>(p));
+}
+__device__ __forceinline__ float4 load4(const __nv_bfloat16 *p) {
+  uint2 r = __ldg(reinterpret_cast<const uint2 *>(p));
+  float4 f;
+  f.x = __uint_as_float(r.x << 16);
+  f.y = __uint_as_float(r.x & 0xffff0000u);
+  f.z = __uint_as_float(r.y << 16);
+  f.w = __uint_as_float(r.y & 0xffff0000u);
+  return f;
+}
+
+__device__ __forceinline__ void store4(float *p, float a, float b, float c, float d) {
+  *reinterpret_cast<float4 *>(p) = make_float4(a, b, c, d);
+}
+__device__ __forceinline__ void store4(__nv_bfloat16 *p, float a, float b, float c, float d) {
+  __nv_bfloat162 lo = __floats2bfloat162_rn(a, b);
+  __nv_bfloat162 hi = __floats2bfloat162_rn(c, d);
+  uint2 r;
+  r.x = *reinterpret_cast<uint32_t *>(&lo);
+  r.y = *reinterpret_cast<uint32_t *>(&hi);
+  *reinterpret_cast<uint2 *>(p) = r;
+}
+
+// --------------------------------------------------------------- codecs ----
+// INT8: c = clamp(rint(x / s), -127, 127); y = c * s.  s > 0.
+__device__ __forceinline__ float qdq_int8(float x, float s) {
+  float c = rintf(__fdiv_rn(x, s));
+  c = fminf(fmaxf(c, -127.0f), 127.0f);
+  return __fmul_rn(c, s);
+}
+
+// E4M3 round trip of two values: RNE with saturation to +-448 (the
+// conversion's satfinite mode), then back to fp32 exactly.
+__device__ __forceinline__ float2 e4m3_round2(float a, float b) {
+  __nv_fp8x2_storage_t p = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+  __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(p, __NV_E4M3);
+  __half2 hh = *reinterpret_cast<__half2 *>(&h);
+  return __half22float2(hh);
+}
+
+// FP8 tile codec for two values sharing scale s > 0.
+__device__ __forceinline__ float2 qdq_fp8_2(float x0, float x1, float s) {
+  float2 c = e4m3_round2(__fdiv_rn(x0, s), __fdiv_rn(x1, s));
+  return make_float2(__fmul_rn(c.x, s), __fmul_rn(c.y, s));
+}
+
+__device__ __forceinline__ float int8_scale(float amax) { return __fdiv_rn(amax, 127.0f); }
+__device__ __forceinline__ float fp8_scale(float amax) { return __fdiv_rn(amax, 448.0f); }
+
+// Reductions over aligned lane groups of size W (power of two <= 32).
+template <int W>
+__device__ __forceinline__ float group_max(float x) {
+#pragma unroll
+  for (int off = 1; off < W; off <<= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, off));
+  return x;
+}
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+  return x;
+}
+
+}  // namespace gdn

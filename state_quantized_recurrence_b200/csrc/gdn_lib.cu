@@ -1,0 +1,202 @@
+// C ABI of the gated-delta-rule library (declared in include/gdn_qdq.h):
+// argument validation on the host, kernel selection, and the per-device
+// error word.  Nothing here computes the method; every arithmetic step runs
+// in the kernels included below.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "gdn_qdq.h"
+#include "gdn_common.cuh"
+#include "gdn_decode.cuh"
+#include "gdn_prefill_simt.cuh"
+
+namespace {
+
+// Per-device error word (bits gdn::kErrBadSeqlens / kErrTimeout), set by
+// kernels with atomicOr and read-and-cleared by gdn_last_error().
+__device__ unsigned g_err_word;
+
+constexpr int kMaxDevices = 64;
+unsigned *g_err_ptr[kMaxDevices];  // device address of g_err_word per device
+
+gdn_status err_word(unsigned **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return GDN_ERR_CUDA;
+  if (!g_err_ptr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_err_word) != cudaSuccess) return GDN_ERR_CUDA;
+    g_err_ptr[dev] = static_cast<unsigned *>(p);
+  }
+  *out = g_err_ptr[dev];
+  return GDN_OK;
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool qdq_params(gdn_qdq_mode m, int d_v, int *kind, int *group) {
+  switch (m) {
+    case GDN_QDQ_NONE: *kind = gdn::kQdqNone; *group = 32; return true;
+    case GDN_QDQ_FP8_E4M3_TILE64: *kind = gdn::kQdqFp8Tile; *group = 64; return d_v % 64 == 0;
+    case GDN_QDQ_INT8_GROUP16: *kind = gdn::kQdqInt8; *group = 16; return true;
+    case GDN_QDQ_INT8_GROUP32: *kind = gdn::kQdqInt8; *group = 32; return true;
+    case GDN_QDQ_INT8_GROUP64: *kind = gdn::kQdqInt8; *group = 64; return true;
+  }
+  return false;
+}
+
+// Shared checks; returns GDN_OK or the status to report.
+// `tokens` is the number of token rows the call reads (0: the token
+// pointers are not used and may be NULL).
+gdn_status check_common(const void *q, const void *k, const void *v, const float *g,
+                        const float *beta, const void *o, int n_seq, int H, int d_k,
+                        int d_v, gdn_dtype dt, gdn_gate_kind gk, gdn_qdq_mode qdq,
+                        long long tokens) {
+  if (n_seq < 0 || H <= 0 || d_k <= 0 || d_v <= 0) return GDN_ERR_INVALID_ARG;
+  if (dt != GDN_DTYPE_BF16 && dt != GDN_DTYPE_F32) return GDN_ERR_UNSUPPORTED;
+  if (gk != GDN_GATE_SCALAR && gk != GDN_GATE_PER_KEY) return GDN_ERR_UNSUPPORTED;
+  if ((unsigned)qdq > (unsigned)GDN_QDQ_INT8_GROUP64) return GDN_ERR_UNSUPPORTED;
+  if ((d_k != 64 && d_k != 128) || (d_v != 64 && d_v != 128)) return GDN_ERR_UNSUPPORTED;
+  if (n_seq == 0 || tokens == 0) return GDN_OK;
+  if (!q || !k || !v || !g || !beta || !o) return GDN_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      !aligned(g, 4) || !aligned(beta, 4))
+    return GDN_ERR_INVALID_ARG;
+  return GDN_OK;
+}
+
+template <typename Tin>
+gdn_status launch_decode(const void *q, const void *k, const void *v, const float *g,
+                         const float *beta, float *state, int n_seq, int H, int d_k,
+                         int d_v, bool per_key, int kind, int group, void *o,
+                         cudaStream_t st) {
+  const long long blocks = (long long)n_seq * H * (d_v / 64);
+  if (blocks > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+  const float scale = (float)(1.0 / sqrt((double)d_k));
+  const Tin *qq = static_cast<const Tin *>(q), *kk = static_cast<const Tin *>(k),
+            *vv = static_cast<const Tin *>(v);
+  Tin *oo = static_cast<Tin *>(o);
+  dim3 grid((unsigned)blocks), block(256);
+#define GDN_DEC(DK, PK) \
+  gdn::decode_kernel<Tin, DK, PK><<<grid, block, 0, st>>>(qq, kk, vv, g, beta, state, oo, d_v, scale, kind, group)
+  if (d_k == 128) { if (per_key) GDN_DEC(128, true); else GDN_DEC(128, false); }
+  else            { if (per_key) GDN_DEC(64, true);  else GDN_DEC(64, false); }
+#undef GDN_DEC
+  return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+template <typename Tin, int DK, bool PK>
+gdn_status launch_simt_one(const Tin *q, const Tin *k, const Tin *v, const float *g,
+                           const float *beta, const float *state_in, const int32_t *cu,
+                           int T, int H, int d_v, float scale, int kind, int group, Tin *o,
+                           float *state_out, unsigned *err, unsigned blocks, cudaStream_t st) {
+  using L = gdn::simt::Smem<DK>;
+  auto kern = gdn::simt::prefill_simt_kernel<Tin, DK, PK>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kBytes) !=
+      cudaSuccess)
+    return GDN_ERR_CUDA;
+  kern<<<blocks, gdn::simt::kThreads, L::kBytes, st>>>(q, k, v, g, beta, state_in, cu, T, H, d_v,
+                                                       scale, kind, group, o, state_out, err);
+  return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+template <typename Tin>
+gdn_status launch_prefill_simt(const void *q, const void *k, const void *v, const float *g,
+                               const float *beta, const float *state_in, const int32_t *cu,
+                               int n_seq, int T, int H, int d_k, int d_v, bool per_key,
+                               int kind, int group, void *o, float *state_out, unsigned *err,
+                               cudaStream_t st) {
+  const long long blocks = (long long)n_seq * H * (d_v / 64);
+  if (blocks > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+  const float scale = (float)(1.0 / sqrt((double)d_k));
+  const Tin *qq = static_cast<const Tin *>(q), *kk = static_cast<const Tin *>(k),
+            *vv = static_cast<const Tin *>(v);
+  Tin *oo = static_cast<Tin *>(o);
+  const unsigned nb = (unsigned)blocks;
+#define GDN_PF(DK, PK) \
+  launch_simt_one<Tin, DK, PK>(qq, kk, vv, g, beta, state_in, cu, T, H, d_v, scale, kind, group, oo, state_out, err, nb, st)
+  if (d_k == 128) return per_key ? GDN_PF(128, true) : GDN_PF(128, false);
+  return per_key ? GDN_PF(64, true) : GDN_PF(64, false);
+#undef GDN_PF
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *gdn_status_string(gdn_status s) {
+  switch (s) {
+    case GDN_OK: return "GDN_OK";
+    case GDN_ERR_INVALID_ARG: return "GDN_ERR_INVALID_ARG";
+    case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED";
+    case GDN_ERR_CUDA: return "GDN_ERR_CUDA";
+    case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT";
+  }
+  return "GDN_ERR_UNKNOWN";
+}
+
+int gdn_version(void) { return 100; }
+
+gdn_status gdn_decode(const void *q, const void *k, const void *v, const float *g,
+                      const float *beta, float *state_inout, int n_seq, int H, int d_k,
+                      int d_v, gdn_dtype dt, gdn_gate_kind gk, gdn_qdq_mode qdq, void *o,
+                      void *cuda_stream) {
+  gdn_status s = check_common(q, k, v, g, beta, o, n_seq, H, d_k, d_v, dt, gk, qdq, n_seq);
+  if (s != GDN_OK) return s;
+  int kind = 0, group = 32;
+  if (!qdq_params(qdq, d_v, &kind, &group)) return GDN_ERR_UNSUPPORTED;
+  if (n_seq == 0) return GDN_OK;
+  if (!state_inout || !aligned(state_inout, 16)) return GDN_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  const bool pk = gk == GDN_GATE_PER_KEY;
+  if (dt == GDN_DTYPE_BF16)
+    return launch_decode<__nv_bfloat16>(q, k, v, g, beta, state_inout, n_seq, H, d_k, d_v, pk,
+                                        kind, group, o, st);
+  return launch_decode<float>(q, k, v, g, beta, state_inout, n_seq, H, d_k, d_v, pk, kind,
+                              group, o, st);
+}
+
+gdn_status gdn_prefill(const void *q, const void *k, const void *v, const float *g,
+                       const float *beta, const float *state_in, const int32_t *cu_seqlens,
+                       int n_seq, int T, int H, int d_k, int d_v, gdn_dtype dt,
+                       gdn_gate_kind gk, gdn_qdq_mode qdq, void *o, float *state_out,
+                       void *cuda_stream) {
+  if (T < 0) return GDN_ERR_INVALID_ARG;
+  const long long rows = cu_seqlens ? (long long)T : (long long)n_seq * T;
+  gdn_status s = check_common(q, k, v, g, beta, o, n_seq, H, d_k, d_v, dt, gk, qdq, rows);
+  if (s != GDN_OK) return s;
+  int kind = 0, group = 32;
+  if (!qdq_params(qdq, d_v, &kind, &group)) return GDN_ERR_UNSUPPORTED;
+  if (n_seq == 0) return GDN_OK;
+  if (!state_out || !aligned(state_out, 16)) return GDN_ERR_INVALID_ARG;
+  if (state_in && !aligned(state_in, 16)) return GDN_ERR_INVALID_ARG;
+  if (cu_seqlens && !aligned(cu_seqlens, 4)) return GDN_ERR_INVALID_ARG;
+  // Total token rows must index within 64-bit element offsets comfortably.
+  if (rows * H * 128 > (1LL << 46)) return GDN_ERR_UNSUPPORTED;
+  unsigned *err = nullptr;
+  if ((s = err_word(&err)) != GDN_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  const bool pk = gk == GDN_GATE_PER_KEY;
+  if (dt == GDN_DTYPE_BF16)
+    return launch_prefill_simt<__nv_bfloat16>(q, k, v, g, beta, state_in, cu_seqlens, n_seq, T,
+                                              H, d_k, d_v, pk, kind, group, o, state_out, err, st);
+  return launch_prefill_simt<float>(q, k, v, g, beta, state_in, cu_seqlens, n_seq, T, H, d_k,
+                                    d_v, pk, kind, group, o, state_out, err, st);
+}
+
+gdn_status gdn_last_error(void *cuda_stream) {
+  unsigned *err = nullptr;
+  gdn_status s = err_word(&err);
+  if (s != GDN_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  unsigned host = 0;
+  if (cudaMemcpyAsync(&host, err, sizeof(unsigned), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return GDN_ERR_CUDA;
+  if (cudaMemsetAsync(err, 0, sizeof(unsigned), st) != cudaSuccess) return GDN_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return GDN_ERR_CUDA;
+  if (host & gdn::kErrTimeout) return GDN_ERR_TIMEOUT;
+  if (host & gdn::kErrBadSeqlens) return GDN_ERR_INVALID_ARG;
+  return GDN_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,444 @@
+// Chunked prefix of the gated delta rule with a QDQ state, fp32 CUDA-core
+// (FFMA) kernel.  It serves the fp32 input dtype, where the tensor-core
+// operand precisions cannot meet a 1e-5 tolerance.
+//
+// Per (sequence, head, 64-column value tile) one CTA walks the sequence in
+// 64-token chunks (PR #2497 What section: "64-token chunks", the
+// "WY-transformed W"; PR #2507 What section: exact triangular solve).  With
+// G_r the within-chunk cumulative log gate (per key channel; a broadcast
+// scalar for GDN), a reference G_ref = G[(n-1)/2] and the factored operands
+//   Kp = K * exp(G - G_ref),  Km = K * exp(G_ref - G),  Qp = Q * exp(G - G_ref)
+// (so Kp_r . Km_i = sum_c k_rc k_ic exp(G_rc - G_ic), bounded for i <= r),
+// one chunk of n <= 64 tokens from state H0 ([d_k, 64] tile) computes
+//   A     = strict_lower(diag(beta) Kp Km^T),  Aqk = lower(Qp Km^T)
+//   [W|U] = (I + A)^-1 [diag(beta) K*exp(G) | diag(beta) V]   (forward subst.)
+//   Vn    = U - W H0
+//   O     = scale * ((Q*exp(G)) H0 + Aqk Vn)
+//   H     = diag(exp(G_n)) H0 + (K*exp(G_n - G))^T Vn
+//   H     = QDQ(H)                                   (every chunk end)
+// Rows past the end of a partial chunk are zero-filled, which makes every
+// product above ignore them without special cases.
+#pragma once
+
+#include "gdn_common.cuh"
+
+namespace gdn {
+namespace simt {
+
+constexpr int kChunk = 64;
+constexpr int kThreads = 256;
+constexpr int LDV = 68;  // row stride (floats) of [64 x 64] tiles
+constexpr int LDA = 66;  // row stride of A / Aqk
+
+template <int DK>
+struct Smem {
+  static constexpr int LDK = DK + 4;
+  static constexpr int kRegion = (64 * LDK > 2 * 64 * LDA) ? 64 * LDK : 2 * 64 * LDA;
+  static constexpr int oK = 0;                     // K -> Kp -> diag(b) K e^G -> W
+  static constexpr int oX = oK + 64 * LDK;         // Km -> Kc = K e^(Gn - G)
+  static constexpr int oQ = oX + 64 * LDK;         // Q -> Qp -> Q e^G
+  static constexpr int oR = oQ + 64 * LDK;         // G (cumsum) -> A | Aqk
+  static constexpr int oV = oR + kRegion;          // V -> diag(b) V -> U -> Vn
+  static constexpr int oH = oV + 64 * LDV;         // state tile [DK x 64]
+  static constexpr int oBeta = oH + DK * LDV;
+  static constexpr int oGs = oBeta + 64;           // scalar-gate cumsum
+  static constexpr int oEref = oGs + 64;           // exp(G_ref)
+  static constexpr int oEn = oEref + DK;           // exp(G_n)
+  static constexpr int oEnr = oEn + DK;            // exp(G_n - G_ref)
+  static constexpr int oGref = oEnr + DK;
+  static constexpr int oGn = oGref + DK;
+  static constexpr int oRed = oGn + DK;
+  static constexpr int kFloats = oRed + 32;
+  static constexpr size_t kBytes = sizeof(float) * kFloats;
+};
+
+__device__ __forceinline__ float dot4(float4 a, float4 b) {
+  return a.x * b.x + a.y * b.y + a.z * b.z + a.w * b.w;
+}
+
+template <typename Tin, int DK, bool PER_KEY>
+__global__ void __launch_bounds__(kThreads, 1)
+prefill_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
+                    const Tin *__restrict__ v, const float *__restrict__ g,
+                    const float *__restrict__ beta,
+                    const float *__restrict__ state_in,
+                    const int *__restrict__ cu_seqlens, int T, int H, int DV,
+                    float scale, int qdq_kind, int qdq_group,
+                    Tin *__restrict__ o, float *__restrict__ state_out,
+                    unsigned *__restrict__ err) {
+  using L = Smem<DK>;
+  constexpr int LDK = L::LDK;
+  extern __shared__ __align__(16) float sm[];
+  float *sK = sm + L::oK, *sX = sm + L::oX, *sQ = sm + L::oQ, *sR = sm + L::oR;
+  float *sA = sR, *sAqk = sR + 64 * LDA;
+  float *sV = sm + L::oV, *sH = sm + L::oH, *sBeta = sm + L::oBeta;
+  float *sGs = sm + L::oGs, *sEref = sm + L::oEref, *sEn = sm + L::oEn;
+  float *sEnr = sm + L::oEnr, *sGref = sm + L::oGref, *sGn = sm + L::oGn;
+  float *sRed = sm + L::oRed;
+
+  const int nvt = DV >> 6;
+  const int vt = blockIdx.x % nvt;
+  const int unit = blockIdx.x / nvt;  // seq * H + head
+  const int h = unit % H, s = unit / H;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int rb = tid >> 4, cb = tid & 15;
+
+  long long t0, t1;
+  if (cu_seqlens) {
+    t0 = cu_seqlens[s];
+    t1 = cu_seqlens[s + 1];
+    const int n_seq = gridDim.x / (H * nvt);
+    if (t0 < 0 || t1 < t0 || t1 > T || (s == 0 && t0 != 0) || (s == n_seq - 1 && t1 != T)) {
+      if (tid == 0) atomicOr(err, kErrBadSeqlens);
+      return;
+    }
+  } else {
+    t0 = (long long)s * T;
+    t1 = t0 + T;
+  }
+  const long long L_seq = t1 - t0;
+
+  // ---- initial state tile ----
+  const long long st_off = (long long)unit * DK * DV + vt * 64;
+  for (int idx = tid; idx < DK * 16; idx += kThreads) {
+    const int r = idx >> 4, c4 = (idx & 15) * 4;
+    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (state_in) x = *reinterpret_cast<const float4 *>(state_in + st_off + (long long)r * DV + c4);
+    *reinterpret_cast<float4 *>(sH + r * LDV + c4) = x;
+  }
+
+  for (long long c0 = 0; c0 < L_seq; c0 += kChunk) {
+    const int n = (int)min((long long)kChunk, L_seq - c0);
+    const long long tb = t0 + c0;
+    __syncthreads();  // previous chunk fully consumed
+
+    // ---- P0: stage the chunk (zero rows past n) ----
+    for (int idx = tid; idx < 64 * (DK / 4); idx += kThreads) {
+      const int r = idx / (DK / 4), c4 = (idx % (DK / 4)) * 4;
+      float4 kx = make_float4(0.f, 0.f, 0.f, 0.f), qx = kx, gx = kx;
+      if (r < n) {
+        const long long off = ((tb + r) * H + h) * DK + c4;
+        kx = load4(k + off);
+        qx = load4(q + off);
+        if (PER_KEY) gx = load4(g + off);
+      }
+      *reinterpret_cast<float4 *>(sK + r * LDK + c4) = kx;
+      *reinterpret_cast<float4 *>(sQ + r * LDK + c4) = qx;
+      if (PER_KEY) *reinterpret_cast<float4 *>(sR + r * LDK + c4) = gx;
+    }
+    for (int idx = tid; idx < 64 * 16; idx += kThreads) {
+      const int r = idx >> 4, c4 = (idx & 15) * 4;
+      float4 vx = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (r < n) vx = load4(v + ((tb + r) * H + h) * DV + vt * 64 + c4);
+      *reinterpret_cast<float4 *>(sV + r * LDV + c4) = vx;
+    }
+    if (tid < 64) {
+      sBeta[tid] = tid < n ? __ldg(beta + (tb + tid) * H + h) : 0.0f;
+      if (!PER_KEY) sGs[tid] = tid < n ? __ldg(g + (tb + tid) * H + h) : 0.0f;
+    }
+    __syncthreads();
+
+    // ---- P1: within-chunk cumulative log gate, reference and end rows ----
+    if (PER_KEY) {
+      if (tid < DK) {
+        float acc = 0.0f;
+        for (int r = 0; r < 64; ++r) {
+          acc += sR[r * LDK + tid];
+          sR[r * LDK + tid] = acc;
+        }
+      }
+    } else if (warp == 0) {
+      float x0 = sGs[lane], x1 = sGs[lane + 32];
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        float y0 = __shfl_up_sync(0xffffffffu, x0, off);
+        float y1 = __shfl_up_sync(0xffffffffu, x1, off);
+        if (lane >= off) { x0 += y0; x1 += y1; }
+      }
+      x1 += __shfl_sync(0xffffffffu, x0, 31);
+      sGs[lane] = x0;
+      sGs[lane + 32] = x1;
+    }
+    __syncthreads();
+    const int rref = (n - 1) >> 1;
+    if (tid < DK) {
+      const float gr = PER_KEY ? sR[rref * LDK + tid] : sGs[rref];
+      const float gn = PER_KEY ? sR[(n - 1) * LDK + tid] : sGs[n - 1];
+      sGref[tid] = gr;
+      sGn[tid] = gn;
+      sEref[tid] = expf(gr);
+      sEn[tid] = expf(gn);
+      sEnr[tid] = expf(gn - gr);
+    }
+    __syncthreads();
+
+    // ---- P2: factored operands Kp, Km, Qp ----
+    for (int idx = tid; idx < 64 * (DK / 4); idx += kThreads) {
+      const int r = idx / (DK / 4), c4 = (idx % (DK / 4)) * 4;
+      float4 kx = *reinterpret_cast<float4 *>(sK + r * LDK + c4);
+      float4 qx = *reinterpret_cast<float4 *>(sQ + r * LDK + c4);
+      float gg[4];
+      if (PER_KEY) {
+        float4 gx = *reinterpret_cast<float4 *>(sR + r * LDK + c4);
+        gg[0] = gx.x; gg[1] = gx.y; gg[2] = gx.z; gg[3] = gx.w;
+      } else {
+        gg[0] = gg[1] = gg[2] = gg[3] = sGs[r];
+      }
+      float ep[4], em[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        ep[e] = expf(gg[e] - sGref[c4 + e]);
+        em[e] = expf(sGref[c4 + e] - gg[e]);
+      }
+      *reinterpret_cast<float4 *>(sK + r * LDK + c4) =
+          make_float4(kx.x * ep[0], kx.y * ep[1], kx.z * ep[2], kx.w * ep[3]);
+      *reinterpret_cast<float4 *>(sX + r * LDK + c4) =
+          make_float4(kx.x * em[0], kx.y * em[1], kx.z * em[2], kx.w * em[3]);
+      *reinterpret_cast<float4 *>(sQ + r * LDK + c4) =
+          make_float4(qx.x * ep[0], qx.y * ep[1], qx.z * ep[2], qx.w * ep[3]);
+    }
+    __syncthreads();
+
+    // ---- P3: A = strict_lower(diag(b) Kp Km^T), Aqk = lower(Qp Km^T) ----
+    {
+      float accA[4][4], accQ[4][4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+#pragma unroll
+        for (int mm = 0; mm < 4; ++mm) accA[m][mm] = accQ[m][mm] = 0.0f;
+      for (int c = 0; c < DK; c += 4) {
+        float4 kp[4], qp[4], km[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          kp[m] = *reinterpret_cast<float4 *>(sK + (rb + 16 * m) * LDK + c);
+          qp[m] = *reinterpret_cast<float4 *>(sQ + (rb + 16 * m) * LDK + c);
+          km[m] = *reinterpret_cast<float4 *>(sX + (cb + 16 * m) * LDK + c);
+        }
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+#pragma unroll
+          for (int mm = 0; mm < 4; ++mm) {
+            accA[m][mm] += dot4(kp[m], km[mm]);
+            accQ[m][mm] += dot4(qp[m], km[mm]);
+          }
+      }
+      __syncthreads();  // the gate cumsum in sR is consumed; A/Aqk overwrite it
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int r = rb + 16 * m;
+        const float br = sBeta[r];
+#pragma unroll
+        for (int mm = 0; mm < 4; ++mm) {
+          const int i = cb + 16 * mm;
+          sA[r * LDA + i] = i < r ? br * accA[m][mm] : 0.0f;
+          sAqk[r * LDA + i] = i <= r ? accQ[m][mm] : 0.0f;
+        }
+      }
+    }
+    __syncthreads();
+
+    // ---- P4: right-hand sides and the remaining scaled operands ----
+    for (int idx = tid; idx < 64 * (DK / 4); idx += kThreads) {
+      const int r = idx / (DK / 4), c4 = (idx % (DK / 4)) * 4;
+      const float br = sBeta[r];
+      float4 kx = *reinterpret_cast<float4 *>(sK + r * LDK + c4);
+      float4 qx = *reinterpret_cast<float4 *>(sQ + r * LDK + c4);
+      float4 mx = *reinterpret_cast<float4 *>(sX + r * LDK + c4);
+      const float e0 = sEref[c4], e1 = sEref[c4 + 1], e2 = sEref[c4 + 2], e3 = sEref[c4 + 3];
+      *reinterpret_cast<float4 *>(sK + r * LDK + c4) =
+          make_float4(br * (kx.x * e0), br * (kx.y * e1), br * (kx.z * e2), br * (kx.w * e3));
+      *reinterpret_cast<float4 *>(sQ + r * LDK + c4) =
+          make_float4(qx.x * e0, qx.y * e1, qx.z * e2, qx.w * e3);
+      *reinterpret_cast<float4 *>(sX + r * LDK + c4) =
+          make_float4(mx.x * sEnr[c4], mx.y * sEnr[c4 + 1], mx.z * sEnr[c4 + 2], mx.w * sEnr[c4 + 3]);
+    }
+    for (int idx = tid; idx < 64 * 16; idx += kThreads) {
+      const int r = idx >> 4, c4 = (idx & 15) * 4;
+      const float br = sBeta[r];
+      float4 vx = *reinterpret_cast<float4 *>(sV + r * LDV + c4);
+      *reinterpret_cast<float4 *>(sV + r * LDV + c4) =
+          make_float4(br * vx.x, br * vx.y, br * vx.z, br * vx.w);
+    }
+    __syncthreads();
+
+    // ---- P5: [W | U] = (I + A)^-1 RHS by forward substitution, one column
+    //      per thread held in registers ----
+    if (tid < DK + 64) {
+      float *colp = tid < DK ? sK + tid : sV + (tid - DK);
+      const int ld = tid < DK ? LDK : LDV;
+      float x[kChunk];
+#pragma unroll
+      for (int r = 0; r < kChunk; ++r) {
+        if (r < n) {
+          float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
+          const float *arow = sA + r * LDA;
+#pragma unroll
+          for (int i = 0; i + 1 < r; i += 2) {
+            float2 aa = *reinterpret_cast<const float2 *>(arow + i);
+            if (i & 2) { p2 += aa.x * x[i]; p3 += aa.y * x[i + 1]; }
+            else       { p0 += aa.x * x[i]; p1 += aa.y * x[i + 1]; }
+          }
+          if (r & 1) p0 += arow[r - 1] * x[r - 1];
+          const float xr = colp[r * ld] - ((p0 + p1) + (p2 + p3));
+          x[r] = xr;
+          colp[r * ld] = xr;
+        } else {
+          x[r] = 0.0f;
+        }
+      }
+    }
+    __syncthreads();
+
+    // ---- P6: Vn = U - W H0 (in place in sV) ----
+    {
+      float acc[4][4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        float4 u4 = *reinterpret_cast<float4 *>(sV + (rb + 16 * m) * LDV + 4 * cb);
+        acc[m][0] = u4.x; acc[m][1] = u4.y; acc[m][2] = u4.z; acc[m][3] = u4.w;
+      }
+      for (int c = 0; c < DK; c += 4) {
+        float4 hh[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) hh[e] = *reinterpret_cast<float4 *>(sH + (c + e) * LDV + 4 * cb);
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          float4 w = *reinterpret_cast<float4 *>(sK + (rb + 16 * m) * LDK + c);
+          const float we[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            acc[m][0] -= we[e] * hh[e].x; acc[m][1] -= we[e] * hh[e].y;
+            acc[m][2] -= we[e] * hh[e].z; acc[m][3] -= we[e] * hh[e].w;
+          }
+        }
+      }
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+        *reinterpret_cast<float4 *>(sV + (rb + 16 * m) * LDV + 4 * cb) =
+            make_float4(acc[m][0], acc[m][1], acc[m][2], acc[m][3]);
+    }
+    __syncthreads();
+
+    // ---- P7: O = scale ((Q e^G) H0 + Aqk Vn) ----
+    {
+      float acc[4][4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[m][e] = 0.0f;
+      for (int c = 0; c < DK; c += 4) {
+        float4 hh[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) hh[e] = *reinterpret_cast<float4 *>(sH + (c + e) * LDV + 4 * cb);
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          float4 qq = *reinterpret_cast<float4 *>(sQ + (rb + 16 * m) * LDK + c);
+          const float qe[4] = {qq.x, qq.y, qq.z, qq.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            acc[m][0] += qe[e] * hh[e].x; acc[m][1] += qe[e] * hh[e].y;
+            acc[m][2] += qe[e] * hh[e].z; acc[m][3] += qe[e] * hh[e].w;
+          }
+        }
+      }
+      for (int i = 0; i < 64; i += 2) {
+        float4 v0 = *reinterpret_cast<float4 *>(sV + i * LDV + 4 * cb);
+        float4 v1 = *reinterpret_cast<float4 *>(sV + (i + 1) * LDV + 4 * cb);
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          float2 aa = *reinterpret_cast<float2 *>(sAqk + (rb + 16 * m) * LDA + i);
+          acc[m][0] += aa.x * v0.x + aa.y * v1.x; acc[m][1] += aa.x * v0.y + aa.y * v1.y;
+          acc[m][2] += aa.x * v0.z + aa.y * v1.z; acc[m][3] += aa.x * v0.w + aa.y * v1.w;
+        }
+      }
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int r = rb + 16 * m;
+        if (r < n)
+          store4(o + ((tb + r) * H + h) * DV + vt * 64 + 4 * cb, scale * acc[m][0],
+                 scale * acc[m][1], scale * acc[m][2], scale * acc[m][3]);
+      }
+    }
+    __syncthreads();
+
+    // ---- P8: H = diag(e^Gn) H0 + Kc^T Vn, then QDQ (P9) ----
+    {
+      constexpr int RPT = DK / 16;  // rows rb*RPT .. +RPT-1, cols 4*cb .. +3
+      float acc[RPT][4];
+#pragma unroll
+      for (int j = 0; j < RPT; ++j) {
+        const int r = rb * RPT + j;
+        float4 h0 = *reinterpret_cast<float4 *>(sH + r * LDV + 4 * cb);
+        const float en = sEn[r];
+        acc[j][0] = en * h0.x; acc[j][1] = en * h0.y; acc[j][2] = en * h0.z; acc[j][3] = en * h0.w;
+      }
+      for (int i = 0; i < 64; ++i) {
+        float4 vn = *reinterpret_cast<float4 *>(sV + i * LDV + 4 * cb);
+#pragma unroll
+        for (int j4 = 0; j4 < RPT; j4 += 4) {
+          float4 kc = *reinterpret_cast<float4 *>(sX + i * LDK + rb * RPT + j4);
+          const float ke[4] = {kc.x, kc.y, kc.z, kc.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            acc[j4 + e][0] += ke[e] * vn.x; acc[j4 + e][1] += ke[e] * vn.y;
+            acc[j4 + e][2] += ke[e] * vn.z; acc[j4 + e][3] += ke[e] * vn.w;
+          }
+        }
+      }
+      if (qdq_kind == kQdqInt8) {
+#pragma unroll
+        for (int j = 0; j < RPT; ++j) {
+          float m = fmaxf(fmaxf(fabsf(acc[j][0]), fabsf(acc[j][1])),
+                          fmaxf(fabsf(acc[j][2]), fabsf(acc[j][3])));
+          for (int off = 1; off < (qdq_group >> 2); off <<= 1)
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+          if (m == 0.0f) {
+            acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
+          } else {
+            const float sc = int8_scale(m);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[j][e] = qdq_int8(acc[j][e], sc);
+          }
+        }
+      } else if (qdq_kind == kQdqFp8Tile) {
+        float m = 0.0f;
+#pragma unroll
+        for (int j = 0; j < RPT; ++j)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) m = fmaxf(m, fabsf(acc[j][e]));
+        m = group_max<32>(m);
+        if (lane == 0) sRed[warp] = m;
+        __syncthreads();
+        m = sRed[0];
+#pragma unroll
+        for (int w = 1; w < 8; ++w) m = fmaxf(m, sRed[w]);
+        if (m == 0.0f) {
+#pragma unroll
+          for (int j = 0; j < RPT; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
+        } else {
+          const float sc = fp8_scale(m);
+#pragma unroll
+          for (int j = 0; j < RPT; ++j) {
+            float2 lo = qdq_fp8_2(acc[j][0], acc[j][1], sc), hi = qdq_fp8_2(acc[j][2], acc[j][3], sc);
+            acc[j][0] = lo.x; acc[j][1] = lo.y; acc[j][2] = hi.x; acc[j][3] = hi.y;
+          }
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < RPT; ++j)
+        *reinterpret_cast<float4 *>(sH + (rb * RPT + j) * LDV + 4 * cb) =
+            make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]);
+    }
+  }
+  __syncthreads();
+
+  // ---- state out ----
+  for (int idx = tid; idx < DK * 16; idx += kThreads) {
+    const int r = idx >> 4, c4 = (idx & 15) * 4;
+    *reinterpret_cast<float4 *>(state_out + st_off + (long long)r * DV + c4) =
+        *reinterpret_cast<float4 *>(sH + r * LDV + c4);
+  }
+}
+
+}  // namespace simt
+}  // namespace gdn

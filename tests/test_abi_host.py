@@ -1,0 +1,127 @@
+"""Host-only checks of the C ABI (no GPU needed, nothing is launched).
+
+* the library loads and exports, unmangled, every function that
+  include/*.h declares;
+* argument errors are caught on the host with the documented status codes
+  before any CUDA call (bad sizes, unsupported d_k / d_v / dtype / gate /
+  codec, null or misaligned pointers);
+* an empty batch (n_seq == 0) is a successful no-op.
+"""
+
+import ctypes
+import glob
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+LIB = os.path.join(ROOT, "state_quantized_recurrence_b200", "libgdn_qdq.so")
+
+OK, INVALID, UNSUPPORTED = 0, 1, 2
+BF16, F32 = 0, 1
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from state_quantized_recurrence_b200 import build
+    build.build()
+    L = ctypes.CDLL(LIB)
+    P, I = ctypes.c_void_p, ctypes.c_int
+    L.gdn_prefill.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P, P, P]
+    L.gdn_prefill.restype = I
+    L.gdn_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, P, P]
+    L.gdn_decode.restype = I
+    L.gdn_status_string.argtypes = [I]
+    L.gdn_status_string.restype = ctypes.c_char_p
+    return L
+
+
+def declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        for m in re.finditer(r"^[A-Za-z_][\w \*]*?\b(gdn_\w+)\s*\(", src, flags=re.M):
+            names.add(m.group(1))
+    return names
+
+
+def test_header_symbols_exported(lib):
+    names = declared_functions()
+    assert {"gdn_prefill", "gdn_decode", "gdn_last_error", "gdn_status_string"} <= names
+    out = subprocess.run(["nm", "-D", "--defined-only", LIB], capture_output=True, text=True,
+                         check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    for n in names:
+        assert n in exported, n
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    assert lib.gdn_status_string(0) == b"GDN_OK"
+    assert lib.gdn_status_string(4) == b"GDN_ERR_TIMEOUT"
+    assert lib.gdn_status_string(99) == b"GDN_ERR_UNKNOWN"
+
+
+A = 0x10000  # a 16-byte aligned stand-in address; never dereferenced
+
+
+def pf(lib, **kw):
+    a = dict(q=A, k=A, v=A, g=A, beta=A, state_in=None, cu=None, n_seq=2, T=64, H=4, d_k=128,
+             d_v=128, dt=BF16, gk=0, qdq=1, o=A, state_out=A, stream=None)
+    a.update(kw)
+    return lib.gdn_prefill(a["q"], a["k"], a["v"], a["g"], a["beta"], a["state_in"], a["cu"],
+                           a["n_seq"], a["T"], a["H"], a["d_k"], a["d_v"], a["dt"], a["gk"],
+                           a["qdq"], a["o"], a["state_out"], a["stream"])
+
+
+def dc(lib, **kw):
+    a = dict(q=A, k=A, v=A, g=A, beta=A, state=A, n_seq=2, H=4, d_k=128, d_v=128, dt=BF16, gk=0,
+             qdq=2, o=A, stream=None)
+    a.update(kw)
+    return lib.gdn_decode(a["q"], a["k"], a["v"], a["g"], a["beta"], a["state"], a["n_seq"],
+                          a["H"], a["d_k"], a["d_v"], a["dt"], a["gk"], a["qdq"], a["o"],
+                          a["stream"])
+
+
+@pytest.mark.parametrize("call", [pf, dc])
+def test_validation_errors(lib, call):
+    assert call(lib, n_seq=-1) == INVALID
+    assert call(lib, H=0) == INVALID
+    assert call(lib, d_k=96) == UNSUPPORTED
+    assert call(lib, d_v=32) == UNSUPPORTED
+    assert call(lib, d_k=256) == UNSUPPORTED
+    assert call(lib, dt=7) == UNSUPPORTED
+    assert call(lib, gk=3) == UNSUPPORTED
+    assert call(lib, qdq=9) == UNSUPPORTED
+    assert call(lib, q=None) == INVALID
+    assert call(lib, beta=None) == INVALID
+    assert call(lib, o=None) == INVALID
+    assert call(lib, k=A + 8) == INVALID          # q/k/v/o need 16-byte alignment
+    assert call(lib, g=A + 2) == INVALID          # g/beta need 4-byte alignment
+    assert call(lib, n_seq=0) == OK               # empty batch: no work, no launch
+
+
+def test_prefill_specific_errors(lib):
+    assert pf(lib, T=-1) == INVALID
+    assert pf(lib, state_out=None) == INVALID
+    assert pf(lib, state_out=A + 4) == INVALID
+    assert pf(lib, state_in=A + 4) == INVALID
+    assert pf(lib, cu=A + 2) == INVALID
+
+
+def test_decode_specific_errors(lib):
+    assert dc(lib, state=None) == INVALID
+    assert dc(lib, state=A + 4) == INVALID
+
+
+def test_binding_refuses_missing_library(tmp_path, monkeypatch):
+    """The binding fails loudly (ImportError) when the CUDA library is absent."""
+    import importlib
+    import state_quantized_recurrence_b200._binding as b
+    monkeypatch.setattr(b, "library_path", str(tmp_path / "missing.so"))
+    with pytest.raises(ImportError):
+        b._load()
+    importlib.reload(b)
