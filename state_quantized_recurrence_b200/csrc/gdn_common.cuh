@@ -54,11 +54,44 @@ __device__ __forceinline__ void store4(__nv_bfloat16 *p, float a, float b, float
 }
 
 // --------------------------------------------------------------- codecs ----
+// Correctly rounded quotient x / s from y = RN(1/s): one product and
+// Markstein's correction step (P. Markstein, "Computation of elementary
+// functions on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1),
+// 1990): with q0 = RN(x*y) within one ulp of x/s, the residual r = x - s*q0 is
+// exact in an FMA and RN(q0 + r*y) = RN(x/s) for normal operands.
+//
+// A scale below 2^-100 (an all-but-zero group or tile) is first multiplied,
+// together with x, by 2^64; power-of-two scaling is exact in both and keeps
+// 1/s finite, so the quotient is unchanged.  Quotients small enough to be
+// subnormal round to code 0 either way.
+struct ScaleRecip {
+  float s;    // the scale itself (dequantization multiplies by it)
+  float pre;  // exact power-of-two pre-scale of x and s (1 or 2^64)
+  float s2;   // s * pre
+  float r;    // RN(1 / s2)
+};
+
+__device__ __forceinline__ ScaleRecip make_scale(float s) {
+  ScaleRecip sr;
+  sr.s = s;
+  sr.pre = s < 0x1p-100f ? 0x1p64f : 1.0f;
+  sr.s2 = __fmul_rn(s, sr.pre);
+  sr.r = __frcp_rn(sr.s2);
+  return sr;
+}
+
+__device__ __forceinline__ float div_by_scale(float x, const ScaleRecip &sr) {
+  const float xs = __fmul_rn(x, sr.pre);
+  const float q0 = __fmul_rn(xs, sr.r);
+  const float r = __fmaf_rn(-q0, sr.s2, xs);
+  return __fmaf_rn(r, sr.r, q0);
+}
+
 // INT8: c = clamp(rint(x / s), -127, 127); y = c * s.  s > 0.
-__device__ __forceinline__ float qdq_int8(float x, float s) {
-  float c = rintf(__fdiv_rn(x, s));
+__device__ __forceinline__ float qdq_int8(float x, const ScaleRecip &sr) {
+  float c = rintf(div_by_scale(x, sr));
   c = fminf(fmaxf(c, -127.0f), 127.0f);
-  return __fmul_rn(c, s);
+  return __fmul_rn(c, sr.s);
 }
 
 // E4M3 round trip of two values: RNE with saturation to +-448 (the
@@ -71,9 +104,9 @@ __device__ __forceinline__ float2 e4m3_round2(float a, float b) {
 }
 
 // FP8 tile codec for two values sharing scale s > 0.
-__device__ __forceinline__ float2 qdq_fp8_2(float x0, float x1, float s) {
-  float2 c = e4m3_round2(__fdiv_rn(x0, s), __fdiv_rn(x1, s));
-  return make_float2(__fmul_rn(c.x, s), __fmul_rn(c.y, s));
+__device__ __forceinline__ float2 qdq_fp8_2(float x0, float x1, const ScaleRecip &sr) {
+  float2 c = e4m3_round2(div_by_scale(x0, sr), div_by_scale(x1, sr));
+  return make_float2(__fmul_rn(c.x, sr.s), __fmul_rn(c.y, sr.s));
 }
 
 __device__ __forceinline__ float int8_scale(float amax) { return __fdiv_rn(amax, 127.0f); }

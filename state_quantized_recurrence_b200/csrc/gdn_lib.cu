@@ -2,14 +2,18 @@
 // argument validation on the host, kernel selection, and the per-device
 // error word.  Nothing here computes the method; every arithmetic step runs
 // in the kernels included below.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
+#include <string.h>
 
 #include "gdn_qdq.h"
 #include "gdn_common.cuh"
 #include "gdn_decode.cuh"
 #include "gdn_prefill_simt.cuh"
+#include "gdn_prefill_tc.cuh"
 
 namespace {
 
@@ -65,6 +69,28 @@ gdn_status check_common(const void *q, const void *k, const void *v, const float
   return GDN_OK;
 }
 
+template <typename Tin, int DK, int DV, bool PK>
+void decode_dispatch(dim3 grid, cudaStream_t st, const Tin *q, const Tin *k, const Tin *v,
+                     const float *g, const float *beta, float *state, Tin *o, float scale,
+                     int kind, int group) {
+#define GDN_DEC(QK, GR) \
+  gdn::decode_kernel<Tin, DK, DV, PK, QK, GR><<<grid, 256, 0, st>>>(q, k, v, g, beta, state, o, scale)
+  if (kind == gdn::kQdqNone) GDN_DEC(gdn::kQdqNone, 32);
+  else if (kind == gdn::kQdqFp8Tile) GDN_DEC(gdn::kQdqFp8Tile, 32);
+  else if (group == 16) GDN_DEC(gdn::kQdqInt8, 16);
+  else if (group == 64) GDN_DEC(gdn::kQdqInt8, 64);
+  else GDN_DEC(gdn::kQdqInt8, 32);
+#undef GDN_DEC
+}
+
+template <typename Tin, int DK, int DV>
+void decode_dispatch_gate(bool per_key, dim3 grid, cudaStream_t st, const Tin *q, const Tin *k,
+                          const Tin *v, const float *g, const float *beta, float *state, Tin *o,
+                          float scale, int kind, int group) {
+  if (per_key) decode_dispatch<Tin, DK, DV, true>(grid, st, q, k, v, g, beta, state, o, scale, kind, group);
+  else decode_dispatch<Tin, DK, DV, false>(grid, st, q, k, v, g, beta, state, o, scale, kind, group);
+}
+
 template <typename Tin>
 gdn_status launch_decode(const void *q, const void *k, const void *v, const float *g,
                          const float *beta, float *state, int n_seq, int H, int d_k,
@@ -76,12 +102,12 @@ gdn_status launch_decode(const void *q, const void *k, const void *v, const floa
   const Tin *qq = static_cast<const Tin *>(q), *kk = static_cast<const Tin *>(k),
             *vv = static_cast<const Tin *>(v);
   Tin *oo = static_cast<Tin *>(o);
-  dim3 grid((unsigned)blocks), block(256);
-#define GDN_DEC(DK, PK) \
-  gdn::decode_kernel<Tin, DK, PK><<<grid, block, 0, st>>>(qq, kk, vv, g, beta, state, oo, d_v, scale, kind, group)
-  if (d_k == 128) { if (per_key) GDN_DEC(128, true); else GDN_DEC(128, false); }
-  else            { if (per_key) GDN_DEC(64, true);  else GDN_DEC(64, false); }
-#undef GDN_DEC
+  dim3 grid((unsigned)blocks);
+#define GDN_DECG(DK, DV) \
+  decode_dispatch_gate<Tin, DK, DV>(per_key, grid, st, qq, kk, vv, g, beta, state, oo, scale, kind, group)
+  if (d_k == 128) { if (d_v == 128) GDN_DECG(128, 128); else GDN_DECG(128, 64); }
+  else            { if (d_v == 128) GDN_DECG(64, 128);  else GDN_DECG(64, 64); }
+#undef GDN_DECG
   return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
@@ -118,6 +144,78 @@ gdn_status launch_prefill_simt(const void *q, const void *k, const void *v, cons
   if (d_k == 128) return per_key ? GDN_PF(128, true) : GDN_PF(128, false);
   return per_key ? GDN_PF(64, true) : GDN_PF(64, false);
 #undef GDN_PF
+}
+
+// ---- tensor-core prefill: TMA descriptors and launch -----------------------
+PFN_cuTensorMapEncodeTiled_v12000 g_encode_tiled = nullptr;
+
+gdn_status encode_fn() {
+  if (g_encode_tiled) return GDN_OK;
+  void *fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+          cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || !fn)
+    return GDN_ERR_CUDA;
+  g_encode_tiled = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  return GDN_OK;
+}
+
+// [rows, H, 128] bf16 viewed as a 3-D tensor; box = 64 columns x 1 head x 64
+// token rows.  Rows past the end of the tensor read as zero.
+gdn_status make_token_map(CUtensorMap *m, const void *ptr, int H, long long rows) {
+  memset(m, 0, sizeof(*m));
+  if (rows <= 0) return GDN_OK;  // no chunk is processed, the map is never used
+  cuuint64_t dims[3] = {128, (cuuint64_t)H, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {128 * 2, (cuuint64_t)H * 128 * 2};
+  cuuint32_t box[3] = {64, 1, 64};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = g_encode_tiled(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr),
+                              dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? GDN_OK : GDN_ERR_CUDA;
+}
+
+template <int QK, int GR>
+gdn_status launch_tc_one(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                         const float *g, const float *beta, const float *state_in,
+                         const int32_t *cu, int T, int H, float scale, __nv_bfloat16 *o,
+                         float *state_out, unsigned *err, unsigned blocks, cudaStream_t st) {
+  auto kern = gdn::tc::prefill_tc_kernel<QK, GR>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)gdn::tc::kSmemBytes) != cudaSuccess)
+    return GDN_ERR_CUDA;
+  kern<<<blocks, gdn::tc::kThreads, gdn::tc::kSmemBytes, st>>>(mq, mk, mv, g, beta, state_in, cu,
+                                                               T, H, scale, o, state_out, err);
+  return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status launch_prefill_tc(const void *q, const void *k, const void *v, const float *g,
+                             const float *beta, const float *state_in, const int32_t *cu,
+                             int n_seq, int T, int H, int kind, int group, void *o,
+                             float *state_out, unsigned *err, cudaStream_t st) {
+  const long long blocks = (long long)n_seq * H;
+  if (blocks > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+  const long long rows = cu ? (long long)T : (long long)n_seq * T;
+  if (rows > 0x7fffffffLL - 64) return GDN_ERR_UNSUPPORTED;
+  gdn_status s = encode_fn();
+  if (s != GDN_OK) return s;
+  CUtensorMap mq, mk, mv;
+  if ((s = make_token_map(&mq, q, H, rows)) != GDN_OK) return s;
+  if ((s = make_token_map(&mk, k, H, rows)) != GDN_OK) return s;
+  if ((s = make_token_map(&mv, v, H, rows)) != GDN_OK) return s;
+  const float scale = (float)(1.0 / sqrt(128.0));
+  __nv_bfloat16 *oo = static_cast<__nv_bfloat16 *>(o);
+  const unsigned nb = (unsigned)blocks;
+#define GDN_TC(QK, GR) \
+  launch_tc_one<QK, GR>(mq, mk, mv, g, beta, state_in, cu, T, H, scale, oo, state_out, err, nb, st)
+  if (kind == gdn::kQdqNone) return GDN_TC(gdn::kQdqNone, 32);
+  if (kind == gdn::kQdqFp8Tile) return GDN_TC(gdn::kQdqFp8Tile, 32);
+  if (group == 16) return GDN_TC(gdn::kQdqInt8, 16);
+  if (group == 64) return GDN_TC(gdn::kQdqInt8, 64);
+  return GDN_TC(gdn::kQdqInt8, 32);
+#undef GDN_TC
 }
 
 }  // namespace
@@ -177,6 +275,13 @@ gdn_status gdn_prefill(const void *q, const void *k, const void *v, const float 
   if ((s = err_word(&err)) != GDN_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
   const bool pk = gk == GDN_GATE_PER_KEY;
+  // Kernel choice by specialisation: bf16 GDN at d_k = d_v = 128 runs on the
+  // tensor cores; fp32 inputs (whose 1e-5 tolerance the fp16 operand splits
+  // cannot promise), per-key (KDA) gates and d = 64 run on the CUDA-core
+  // kernel.  Both compute the same chunked algebra.
+  if (dt == GDN_DTYPE_BF16 && !pk && d_k == 128 && d_v == 128)
+    return launch_prefill_tc(q, k, v, g, beta, state_in, cu_seqlens, n_seq, T, H, kind, group, o,
+                             state_out, err, st);
   if (dt == GDN_DTYPE_BF16)
     return launch_prefill_simt<__nv_bfloat16>(q, k, v, g, beta, state_in, cu_seqlens, n_seq, T,
                                               H, d_k, d_v, pk, kind, group, o, state_out, err, st);

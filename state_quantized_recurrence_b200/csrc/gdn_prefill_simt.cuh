@@ -395,9 +395,9 @@ prefill_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
           if (m == 0.0f) {
             acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
           } else {
-            const float sc = int8_scale(m);
+            const ScaleRecip sr = make_scale(int8_scale(m));
 #pragma unroll
-            for (int e = 0; e < 4; ++e) acc[j][e] = qdq_int8(acc[j][e], sc);
+            for (int e = 0; e < 4; ++e) acc[j][e] = qdq_int8(acc[j][e], sr);
           }
         }
       } else if (qdq_kind == kQdqFp8Tile) {
@@ -416,10 +416,11 @@ prefill_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
 #pragma unroll
           for (int j = 0; j < RPT; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
         } else {
-          const float sc = fp8_scale(m);
+          const ScaleRecip sr = make_scale(fp8_scale(m));
 #pragma unroll
           for (int j = 0; j < RPT; ++j) {
-            float2 lo = qdq_fp8_2(acc[j][0], acc[j][1], sc), hi = qdq_fp8_2(acc[j][2], acc[j][3], sc);
+            float2 lo = qdq_fp8_2(acc[j][0], acc[j][1], sr);
+            float2 hi = qdq_fp8_2(acc[j][2], acc[j][3], sr);
             acc[j][0] = lo.x; acc[j][1] = lo.y; acc[j][2] = hi.x; acc[j][3] = hi.y;
           }
         }

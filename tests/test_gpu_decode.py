@@ -155,3 +155,22 @@ def test_decode_single_head_edge(cuda_lib):
     b = float(inp["dec_beta"][0, 0, 0])
     np.testing.assert_allclose(S[0, 0].cpu().double().numpy(), np.outer(k, b * v),
                                rtol=1e-5, atol=1e-7)
+
+
+@pytest.mark.parametrize("mode", ["int8_g32", "fp8_tile64"])
+def test_decode_codec_bit_exact_wide_range(cuda_lib, mode):
+    """4 M state values whose groups span 2^-140 .. 2^60 in magnitude: the
+    codec (scale, quotient, rounding, dequantization) is bit-exact against
+    the oracle's IEEE fp32 codec everywhere, tiny scales included."""
+    gen = torch.Generator().manual_seed(123)
+    N, H, dk, dv = 16, 16, 128, 128
+    st = torch.randn((N, H, dk, dv), generator=gen)
+    expo = torch.randint(-140, 60, (N, H, dk, dv // 32), generator=gen).float()
+    st = (st * torch.exp2(expo).repeat_interleave(32, dim=-1)).float()
+    q = torch.randn((N, H, dk), generator=gen).to(torch.bfloat16)
+    v = torch.randn((N, H, dv), generator=gen).to(torch.bfloat16)
+    S = st.cuda()
+    cuda_lib.gdn_decode(q.cuda(), q.cuda(), v.cuda(), torch.zeros((N, H), device="cuda"),
+                        torch.zeros((N, H), device="cuda"), S, qdq=mode)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(S.cpu().numpy(), oracle.qdq(st.numpy(), mode)[0])
