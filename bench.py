@@ -22,6 +22,7 @@ codecs) on a bounded sample of the same workload on the host cores.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -47,6 +48,25 @@ def load_peaks() -> dict:
         return d
     except (OSError, ValueError):
         return dict(FALLBACK_PEAKS)
+
+
+def kernel_source_hash() -> str:
+    """Hash of the CUDA sources; recorded DRAM traffic is valid only for it."""
+    import glob
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "state_quantized_recurrence_b200", "csrc", "*"))):
+        h.update(open(f, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str):
+    """Per-launch DRAM bytes (read + write) of `kernel` on the full workload,
+    from profiles/traffic.json, or None if absent or taken on other sources."""
+    try:
+        rec = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))[kernel]
+    except (OSError, ValueError, KeyError):
+        return None
+    return rec.get("bytes_per_launch") if rec.get("source_hash") == kernel_source_hash() else None
 
 
 # ------------------------------------------------------------ workload math
@@ -218,10 +238,17 @@ def run_ours(args, dist: Dist) -> dict:
     stream = torch.cuda.current_stream(dev)
     sampler = ClockSampler(dist.local)
 
+    if args.only == "decode":  # profiler captures of the decode kernel alone
+        dec = run_decode(args, dist, dev, stream, sampler, peaks)
+        sampler.stop()
+        dist.close()
+        return {"metric": dec["metric"], "value": dec["value"], "unit": dec["unit"],
+                "n_gpus": dist.world, "impl": "ours", "decode": dec}
+
     # ---------------- prefill (headline) ----------------
     case = gs.CONFIGS["gdn_prefill"]
-    if args.small:
-        case = gs.small_case("gdn_prefill", n_seq=1, H=16, T=1024)
+    if args.small:  # same CTA count (B*H = 64), 8 chunks: for profiler captures
+        case = gs.small_case("gdn_prefill", T=512)
     inp = gs.generate(case)
     d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
     o = torch.empty(d["v"].shape, dtype=d["q"].dtype, device=dev)
@@ -258,7 +285,8 @@ def run_ours(args, dist: Dist) -> dict:
     gbs = nbytes / (ms / 1e3) / 1e9
     tfs = flops / (ms / 1e3) / 1e12
     roofline = {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
-                "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": None,
+                "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
+                "traffic": None if args.small else recorded_traffic("prefill_tc"),
                 "kernel": "prefill (one launch per step)", "bytes_per_launch": nbytes,
                 "peak_source": peaks["source"],
                 "tensor": {"achieved": round(tfs, 2), "peak": peaks["bf16_tflops"],
@@ -266,38 +294,13 @@ def run_ours(args, dist: Dist) -> dict:
                            "flops_per_launch": flops}}
 
     # e2e through the C ABI from pinned host buffers (copies inside the timed region)
-    host = {k: d[k].cpu().pin_memory() for k in ("q", "k", "v", "g", "beta")}
-    o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-    st_h = torch.empty(st.shape, dtype=st.dtype).pin_memory()
-    e2e_steps = max(3, min(args.steps, 10))
-
-    def e2e_step():
-        for k in host:
-            d[k].copy_(host[k], non_blocking=True)
-        step()
-        o_h.copy_(o, non_blocking=True)
-        st_h.copy_(st, non_blocking=True)
-
-    e2e_step()
-    torch.cuda.synchronize(dev)
-    dist.barrier()
-    ev0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    ev1.record(stream)
-    torch.cuda.synchronize(dev)
-    dist.barrier()
-    ms_e2e = dist.max(ev0.elapsed_time(ev1) / e2e_steps)
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = o_h.numel() * o_h.element_size() + st_h.numel() * st_h.element_size()
-    e2e = {"value": dist.world * tokens / (ms_e2e / 1e3), "unit": "tokens/s",
-           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_e2e, 4),
-           "steps": e2e_steps}
-
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, dist, d, o, st, step, stream, tokens)
     cpu = None
     if dist.world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline_prefill(case, inp)
-    del d, host, o, st, o_h, st_h
+    del d, o, st
     torch.cuda.empty_cache()
 
     # ---------------- decode ----------------
@@ -323,6 +326,41 @@ def run_ours(args, dist: Dist) -> dict:
     return res
 
 
+def run_e2e(args, dist, d, o, st, step, stream, tokens) -> dict:
+    """The headline metric through the C ABI with the step's inputs copied
+    from pinned host memory and its outputs read back, inside the timed region."""
+    import torch
+    host = {k: d[k].cpu().pin_memory() for k in ("q", "k", "v", "g", "beta")}
+    o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    st_h = torch.empty(st.shape, dtype=st.dtype).pin_memory()
+    e2e_steps = max(3, min(args.steps, 10))
+
+    def e2e_step():
+        for k in host:
+            d[k].copy_(host[k], non_blocking=True)
+        step()
+        o_h.copy_(o, non_blocking=True)
+        st_h.copy_(st, non_blocking=True)
+
+    e2e_step()
+    dev = o.device
+    torch.cuda.synchronize(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    ev0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    ms_e2e = dist.max(ev0.elapsed_time(ev1) / e2e_steps)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = o_h.numel() * o_h.element_size() + st_h.numel() * st_h.element_size()
+    return {"value": dist.world * tokens / (ms_e2e / 1e3), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": round(ms_e2e, 4), "steps": e2e_steps}
+
+
 def run_decode(args, dist, dev, stream, sampler, peaks) -> dict:
     import torch
 
@@ -330,7 +368,7 @@ def run_decode(args, dist, dev, stream, sampler, peaks) -> dict:
     import state_quantized_recurrence_b200 as sqr
 
     case = gs.CONFIGS["serving_decode"]
-    if args.small:
+    if args.small:  # 64 x 32 heads (134 MB of state > L2), 16 tokens: for profiler captures
         case = gs.small_case("serving_decode", n_seq=64, decode_steps=16)
     inp = gs.generate(case)
     S_steps = case.decode_steps
@@ -385,7 +423,8 @@ def run_decode(args, dist, dev, stream, sampler, peaks) -> dict:
             "ms_per_token_step": round(ms_tok, 5), "reps": reps,
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
-                         "traffic": None, "bytes_per_update": bpu,
+                         "traffic": None if args.small else recorded_traffic("decode"),
+                         "bytes_per_update": bpu, "bytes_per_launch": case.n_seq * case.H * bpu,
                          "peak_source": peaks["source"]},
             "gpu_launches": S_steps * reps, "clocks": sampler.summary(t_wall0, t_wall1),
             "cpu_baseline": cpu}
@@ -440,9 +479,14 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--only", choices=["prefill", "decode"], default=None,
+                    help="measure one kernel only (profiler captures)")
+    ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--small", action="store_true", help="small case (profiling captures)")
     args = ap.parse_args()
+    if args.only == "prefill":
+        args.no_decode = True
     if args.warmup < 3 and not args.small:
         raise SystemExit("--warmup must be >= 3")
     dist = Dist(args.gpus)

@@ -162,8 +162,9 @@ gdn_status encode_fn() {
 }
 
 // [rows, H, 128] bf16 viewed as a 3-D tensor; box = 64 columns x 1 head x 64
-// token rows.  Rows past the end of the tensor read as zero.
-gdn_status make_token_map(CUtensorMap *m, const void *ptr, int H, long long rows) {
+// token rows (128-byte rows, optionally 128B-swizzled into the layout the
+// tensor cores read).  Rows past the end of the tensor read as zero.
+gdn_status make_token_map(CUtensorMap *m, const void *ptr, int H, long long rows, bool swizzle) {
   memset(m, 0, sizeof(*m));
   if (rows <= 0) return GDN_OK;  // no chunk is processed, the map is never used
   cuuint64_t dims[3] = {128, (cuuint64_t)H, (cuuint64_t)rows};
@@ -172,7 +173,8 @@ gdn_status make_token_map(CUtensorMap *m, const void *ptr, int H, long long rows
   cuuint32_t es[3] = {1, 1, 1};
   CUresult r = g_encode_tiled(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr),
                               dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                              swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? GDN_OK : GDN_ERR_CUDA;
 }
@@ -202,9 +204,9 @@ gdn_status launch_prefill_tc(const void *q, const void *k, const void *v, const 
   gdn_status s = encode_fn();
   if (s != GDN_OK) return s;
   CUtensorMap mq, mk, mv;
-  if ((s = make_token_map(&mq, q, H, rows)) != GDN_OK) return s;
-  if ((s = make_token_map(&mk, k, H, rows)) != GDN_OK) return s;
-  if ((s = make_token_map(&mv, v, H, rows)) != GDN_OK) return s;
+  if ((s = make_token_map(&mq, q, H, rows, true)) != GDN_OK) return s;
+  if ((s = make_token_map(&mk, k, H, rows, true)) != GDN_OK) return s;
+  if ((s = make_token_map(&mv, v, H, rows, false)) != GDN_OK) return s;
   const float scale = (float)(1.0 / sqrt(128.0));
   __nv_bfloat16 *oo = static_cast<__nv_bfloat16 *>(o);
   const unsigned nb = (unsigned)blocks;

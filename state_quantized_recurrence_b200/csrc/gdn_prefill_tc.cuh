@@ -16,17 +16,29 @@
 //   H     = gamma_n H0 + K^T diag(exp(G_n - G_t)) Vn,   H = QDQ(H)
 //
 // Every product is issued transposed so that its M side is 128 (the value or
-// key axis): [K;Q] K^T, H0^T [K;Q]^T, R^T T^T, Vn^T Aqk^T and K^T (dVn) each
-// have M = 128.  Operands are fp16 in 128-byte-swizzled shared memory tiles;
-// q/k/v (bf16) convert exactly for |x| in the fp16 range, the codes of a QDQ'd
-// state are exact, and fp32 operands that are not exact (H0, R, T, dVn) are
-// split into hi + lo fp16 pairs (about 22 significant bits), so the state
-// chain keeps near-fp32 accuracy; output-only terms use the hi part.
+// key axis): [K;Q] K^T, H0^T [K;Q]^T, R^T T^T, Vn^T Aqk^T and K^T (dVn).  The
+// A operands R^T and Vn^T go to TMEM (their epilogue thread already owns the
+// row); the rest are fp16 in 128-byte-swizzled shared-memory tiles.  q/k
+// arrive by TMA (bf16, swizzled) into a double buffer and are converted to
+// fp16 in place (exact for |x| in the fp16 range).  Non-exact fp32 operands
+// (H0, R, T, dVn) are split into hi + lo fp16 pairs (about 22 significant
+// bits); with FP8 QDQ the state after the first boundary is exactly
+// E4M3 code x tile scale, so H0 enters as one exact fp16 term and the scale
+// is applied to the product.  Output-only terms use the hi part.
 //
-// Roles: warps 0-3 own TMEM lanes 0-127 and run every accumulator epilogue;
-// all 8 warps convert inputs and run the triangular solve; thread 0 issues
-// TMA loads and MMAs.  Every mbarrier wait is bounded; on a timeout the CTA
-// records kErrTimeout, stops, releases its TMEM and returns.
+// Schedule of one chunk c (256 threads, warpgroups WG0 = warps 0-3 and
+// WG1 = warps 4-7, both covering TMEM lanes 0-127):
+//   MMA2(c)                       [thread 0]
+//   WG0: A, Aqk from MMA1(c); triangular solve; T hi/lo
+//   WG1: R = beta (V - gamma P) -> TMEM; next gates; convert chunk c+1's
+//        [K;Q] in place and issue MMA1(c+1)
+//   MMA3(c): Vn^T = R^T T^T       [thread 0]
+//   all: Vn^T -> TMEM, dVn^T hi/lo -> shared memory
+//   MMA4(c): (Aqk Vn)^T, MMA5(c): H += K^T dVn   [thread 0]
+//   all: outputs, state QDQ (each warpgroup one 64-column tile), H0 operands;
+//        prefetch chunk c+2 into the buffer chunk c released
+// Every mbarrier wait is bounded; on a timeout the CTA records kErrTimeout,
+// stops, lets its in-flight TMA loads land, releases its TMEM and returns.
 #pragma once
 
 #include "gdn_common.cuh"
@@ -41,33 +53,51 @@ constexpr int kD = 128;     // d_k = d_v
 constexpr uint64_t kWaitNs = 2000000000ull;  // bounded waits give up after 2 s
 
 // Shared-memory map (byte offsets from a 1024-byte aligned base).
-constexpr uint32_t OFF_KQ = 0;          // [K;Q] fp16, 2 blocks x [128 rows x 128 B]
-constexpr uint32_t OFF_H = 32768;       // H0 hi (2 blocks), lo (2 blocks): [k][v]
-constexpr uint32_t OFF_X = 98304;       // 48 KB, reused within a chunk (see below)
-constexpr uint32_t OFF_AQK = 147456;    // Aqk fp16 [64 x 64]
-constexpr uint32_t OFF_STG = 155648;    // TMA staging: Q0 Q1 K0 K1 V0 V1 (8 KB each)
-constexpr uint32_t OFF_SMALL = 204800;  // gates, flags, barriers
-constexpr uint32_t kSmemBytes = OFF_SMALL + 2048 + 1024;  // + alignment slack
-// Region X, first half of a chunk:  R^T hi [0,16K) | R^T lo [16K,32K) |
-//   T hi [32K,40K) | T lo [40K,48K); the solve uses A fp32 at [0, 16640) and
-//   its partial products at [16640, 29120) before R^T is written.
-// Region X, second half: Vn^T hi [0,16K) | dVn^T hi [16K,32K) | dVn^T lo [32K,48K).
-constexpr uint32_t X_RHI = 0, X_RLO = 16384, X_THI = 32768, X_TLO = 40960;
-constexpr uint32_t X_VN = 0, X_DVHI = 16384, X_DVLO = 32768;
-constexpr uint32_t X_A32 = 0, X_P32 = 16640;
-constexpr int LDS = 65;  // fp32 row stride of the solve's matrices
+constexpr uint32_t OFF_KQ = 0;          // 2 buffers x [K;Q]: 2 blocks x [128 rows x 128 B]
+constexpr uint32_t OFF_H = 65536;       // H0 hi (2 blocks), lo (2 blocks): [k][v]
+constexpr uint32_t OFF_X = 131072;      // 32 KB, reused within a chunk (below)
+constexpr uint32_t OFF_AQK = 163840;    // Aqk fp16 [64 x 64]
+constexpr uint32_t OFF_V = 172032;      // V staging (TMA, bf16): 2 x [64 tok x 64 v]
+constexpr int LDT = 68;                 // fp32 row stride of the solve's matrices
+constexpr uint32_t OFF_P = 188416;      // solve partial products fp32 [32 x LDT]
+constexpr uint32_t OFF_T = OFF_P + 32 * LDT * 4;  // solve T fp32 [64 x LDT]
+constexpr uint32_t OFF_SMALL = OFF_T + 64 * LDT * 4;  // gates, flags, barriers
+constexpr uint32_t kSmemBytes = OFF_SMALL + 4096 + 1024;  // + alignment slack
+// Region X: first half of a chunk: A fp32 [64 x LDT] at [0, 17408) (its last
+// row overlaps T hi, which is written only after the solve has read A), T hi
+// at [16K,24K), T lo at [24K,32K); second half: dVn^T hi [0,16K), lo [16K,32K).
+constexpr uint32_t X_A = 0, X_THI = 16384, X_TLO = 24576, X_DVHI = 0, X_DVLO = 16384;
 // TMEM columns.
-constexpr uint32_t TM_D1 = 0, TM_D2 = 64, TM_D3 = 192, TM_D4 = 256, TM_COLS = 512;
+constexpr uint32_t TM_D1 = 0;     // [K;Q] K^T               128 x 64 fp32
+constexpr uint32_t TM_D2 = 64;    // P^T | O^T accumulator    128 x 128 fp32
+constexpr uint32_t TM_D3 = 192;   // Vn^T                     128 x 64 fp32
+constexpr uint32_t TM_D4 = 256;   // H [k][v]                 128 x 128 fp32
+constexpr uint32_t TM_RHI = 384;  // R^T hi as A operand      128 x 64 fp16
+constexpr uint32_t TM_RLO = 416;  // R^T lo
+constexpr uint32_t TM_D5 = 384;   // (Aqk Vn)^T, after MMA 3  128 x 64 fp32
+constexpr uint32_t TM_VN = 448;   // Vn^T hi as A operand     128 x 64 fp16
+constexpr uint32_t TM_COLS = 512;
+
+// 16-byte aligned so that both buffers of Small::gt allow float4 loads.
+struct __align__(16) Gates {
+  float G[64], beta[64], gam[64], dec[64], ep[64], em[64];
+  float gn_exp;  // exp(G_{n-1}): decay of the chunk-start state over the chunk
+  int direct;    // 1: per-element exp of gate differences (wide gate span)
+};
 
 struct Small {
-  float G[64], beta[64], gam[64], dec[64], ep[64], em[64];
-  float red[8];
-  float gn_exp;
-  int direct;  // 1: per-element exp of gate differences (wide gate span)
+  Gates gt[2];      // gates of the current and the next chunk
+  float red[2][4];  // FP8 tile amax partials per warpgroup
+  float hs[2];      // FP8 tile scales of H0 when `exact`
+  int exact;        // H0 operand holds exact codes (FP8, after a boundary)
   int abort;
+  int qk_pend[2], v_pend;  // 1 + parity of an issued, unconsumed TMA phase
   uint32_t tmem;
-  uint64_t bar_qk, bar_v, bar_m1, bar_m2, bar_m3, bar_m4;
+  uint64_t bar_qk[2], bar_v, bar_m1, bar_m2, bar_m3, bar_m4;
 };
+static_assert(sizeof(Small) <= 4096, "small-state block overflows its slot");
+static_assert(sizeof(Gates) % 16 == 0 && OFF_SMALL % 16 == 0, "gate arrays must stay 16-byte aligned");
+static_assert(OFF_P % 16 == 0 && OFF_T % 16 == 0 && (LDT * 4) % 16 == 0, "float4 rows");
 
 // Byte address of 16-byte chunk `ch` of row `r` in a 128B-swizzled tile.
 __device__ __forceinline__ uint32_t sw128(uint32_t tile, int r, int ch) {
@@ -101,28 +131,39 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
   return v;
 }
 
-// Write 64 fp32 values of one tile row as fp16 (hi only) into a [rows x 64]
-// 128B-swizzled tile.
-__device__ __forceinline__ void store_row_h(uint32_t tile, int r, const float *x) {
+// 32 fp32 values -> chunks ch0 .. ch0+3 of row r of a hi and a lo tile.
+__device__ __forceinline__ void store32_hl(uint32_t thi, uint32_t tlo, int r, int ch0,
+                                           const float *x) {
 #pragma unroll
-  for (int ch = 0; ch < 8; ++ch)
-    st_shared_v4(sw128(tile, r, ch), pack_h2(x[8 * ch], x[8 * ch + 1]),
-                 pack_h2(x[8 * ch + 2], x[8 * ch + 3]), pack_h2(x[8 * ch + 4], x[8 * ch + 5]),
-                 pack_h2(x[8 * ch + 6], x[8 * ch + 7]));
+  for (int c = 0; c < 4; ++c) {
+    uint32_t h0, h1, h2, h3, l0, l1, l2, l3;
+    split_h2(x[8 * c], x[8 * c + 1], h0, l0);
+    split_h2(x[8 * c + 2], x[8 * c + 3], h1, l1);
+    split_h2(x[8 * c + 4], x[8 * c + 5], h2, l2);
+    split_h2(x[8 * c + 6], x[8 * c + 7], h3, l3);
+    st_shared_v4(sw128(thi, r, ch0 + c), h0, h1, h2, h3);
+    st_shared_v4(sw128(tlo, r, ch0 + c), l0, l1, l2, l3);
+  }
 }
 
-// Same, split into hi and lo tiles.
-__device__ __forceinline__ void store_row_hl(uint32_t thi, uint32_t tlo, int r, const float *x) {
-#pragma unroll
-  for (int ch = 0; ch < 8; ++ch) {
-    uint32_t h0, h1, h2, h3, l0, l1, l2, l3;
-    split_h2(x[8 * ch], x[8 * ch + 1], h0, l0);
-    split_h2(x[8 * ch + 2], x[8 * ch + 3], h1, l1);
-    split_h2(x[8 * ch + 4], x[8 * ch + 5], h2, l2);
-    split_h2(x[8 * ch + 6], x[8 * ch + 7], h3, l3);
-    st_shared_v4(sw128(thi, r, ch), h0, h1, h2, h3);
-    st_shared_v4(sw128(tlo, r, ch), l0, l1, l2, l3);
-  }
+// E4M3 codes of x0/s2 and x1/s2 (correctly rounded quotients from r = RN(1/s2),
+// Markstein's correction), returned as an fp16 pair (exact); y0, y1 receive
+// the dequantized values code * s (s = s2 unless the operands were
+// pre-scaled by a power of two).
+__device__ __forceinline__ uint32_t fp8_code_pair(float x0, float x1, float s2, float r, float &y0,
+                                                  float &y1, float s = 0.0f) {
+  const float q0 = __fmul_rn(x0, r), q1 = __fmul_rn(x1, r);
+  const float t0 = __fmaf_rn(__fmaf_rn(-q0, s2, x0), r, q0);
+  const float t1 = __fmaf_rn(__fmaf_rn(-q1, s2, x1), r, q1);
+  const __nv_fp8x2_storage_t f8 =
+      __nv_cvt_float2_to_fp8x2(make_float2(t0, t1), __NV_SATFINITE, __NV_E4M3);
+  const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(f8, __NV_E4M3);
+  const __half2 hh = *reinterpret_cast<const __half2 *>(&hr);
+  const float2 cf = __half22float2(hh);
+  const float sd = s == 0.0f ? s2 : s;
+  y0 = __fmul_rn(cf.x, sd);
+  y1 = __fmul_rn(cf.y, sd);
+  return *reinterpret_cast<const uint32_t *>(&hh);
 }
 
 __device__ __forceinline__ uint64_t kdesc(uint32_t addr) {
@@ -133,11 +174,71 @@ __device__ __forceinline__ uint64_t mndesc(uint32_t addr, uint32_t lbo) {
 }
 
 // Bounded wait by every calling thread; a timeout marks the CTA aborted.
-__device__ __forceinline__ void wait_or_abort(uint64_t *bar, uint32_t parity, Small *sm,
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, Small *sm,
                                               unsigned *err) {
   if (!sm100::mbar_wait(bar, parity, kWaitNs)) {
     sm->abort = 1;
     atomicOr(err, kErrTimeout);
+    return false;
+  }
+  return true;
+}
+
+// Gates of one chunk (one warp): G = inclusive cumsum of the log gates,
+// gamma = exp(G), dec = exp(G_{n-1} - G), the factors exp(+-(G - G_ref))
+// around the middle token, and beta; rows past n are zero-gated.
+__device__ __forceinline__ void load_gates(Gates *gt, const float *__restrict__ g,
+                                           const float *__restrict__ beta, long long tb, int n,
+                                           int H, int h, int lane) {
+  float x0 = lane < n ? __ldg(g + (tb + lane) * H + h) : 0.0f;
+  float x1 = lane + 32 < n ? __ldg(g + (tb + lane + 32) * H + h) : 0.0f;
+  gt->beta[lane] = lane < n ? __ldg(beta + (tb + lane) * H + h) : 0.0f;
+  gt->beta[lane + 32] = lane + 32 < n ? __ldg(beta + (tb + lane + 32) * H + h) : 0.0f;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const float y0 = __shfl_up_sync(0xffffffffu, x0, off);
+    const float y1 = __shfl_up_sync(0xffffffffu, x1, off);
+    if (lane >= off) { x0 += y0; x1 += y1; }
+  }
+  x1 += __shfl_sync(0xffffffffu, x0, 31);
+  const int rref = (n - 1) >> 1;
+  const float gref = __shfl_sync(0xffffffffu, rref < 32 ? x0 : x1, rref & 31);
+  const float gn = __shfl_sync(0xffffffffu, (n - 1) < 32 ? x0 : x1, (n - 1) & 31);
+  const float g0 = __shfl_sync(0xffffffffu, x0, 0);
+  gt->G[lane] = x0;
+  gt->G[lane + 32] = x1;
+  gt->gam[lane] = expf(x0);
+  gt->gam[lane + 32] = expf(x1);
+  gt->dec[lane] = expf(gn - x0);
+  gt->dec[lane + 32] = expf(gn - x1);
+  gt->ep[lane] = expf(x0 - gref);
+  gt->ep[lane + 32] = expf(x1 - gref);
+  gt->em[lane] = expf(gref - x0);
+  gt->em[lane + 32] = expf(gref - x1);
+  if (lane == 0) {
+    gt->gn_exp = expf(gn);
+    gt->direct = (g0 - gref > 80.0f || gref - gn > 80.0f) ? 1 : 0;
+  }
+}
+
+// In-place bf16 -> fp16 conversion of one [K;Q] buffer (16-byte chunks in
+// their swizzled positions); rows of tokens past n are zeroed.  `nthr`
+// threads, this one being `t`.
+__device__ __forceinline__ void convert_kq(uint32_t buf, int n, int t, int nthr) {
+  for (int e = t; e < 2048; e += nthr) {
+    const int blk = e >> 10, rw = (e >> 3) & 127, ch = e & 7;
+    const uint32_t addr = buf + (uint32_t)blk * 16384u + (uint32_t)rw * 128u + (uint32_t)ch * 16u;
+    uint4 w = make_uint4(0u, 0u, 0u, 0u);
+    if ((rw & 63) < n) {
+      const uint4 src = ld_shared_v4(addr);
+      const uint32_t in[4] = {src.x, src.y, src.z, src.w};
+      uint32_t outw[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        outw[j] = pack_h2(__uint_as_float(in[j] << 16), __uint_as_float(in[j] & 0xffff0000u));
+      w = make_uint4(outw[0], outw[1], outw[2], outw[3]);
+    }
+    st_shared_v4(addr, w.x, w.y, w.z, w.w);
   }
 }
 
@@ -154,12 +255,14 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   const uint32_t base = (raw_addr + 1023u) & ~1023u;
   uint8_t *gbase = smem_raw + (base - raw_addr);
   Small *sm = reinterpret_cast<Small *>(gbase + OFF_SMALL);
-  float *sA = reinterpret_cast<float *>(gbase + OFF_X + X_A32);
-  float *sP = reinterpret_cast<float *>(gbase + OFF_X + X_P32);
-  float *sT = reinterpret_cast<float *>(gbase + OFF_STG);  // solve output, fp32 [64][LDS]
+  float *sA = reinterpret_cast<float *>(gbase + OFF_X + X_A);
+  float *sP = reinterpret_cast<float *>(gbase + OFF_P);
+  float *sT = reinterpret_cast<float *>(gbase + OFF_T);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int unit = blockIdx.x;  // seq * H + head
+  const int wg = warp >> 2;                // warpgroup
+  const int row = 32 * (warp & 3) + lane;  // TMEM lane = accumulator row
+  const int unit = blockIdx.x;             // seq * H + head
   const int h = unit % H, s = unit / H;
 
   long long t0, t1;
@@ -188,7 +291,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   }
 
   if (tid == 0) {
-    sm100::mbar_init(&sm->bar_qk, 1);
+    sm100::mbar_init(&sm->bar_qk[0], 1);
+    sm100::mbar_init(&sm->bar_qk[1], 1);
     sm100::mbar_init(&sm->bar_v, 1);
     sm100::mbar_init(&sm->bar_m1, 1);
     sm100::mbar_init(&sm->bar_m2, 1);
@@ -196,469 +300,542 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     sm100::mbar_init(&sm->bar_m4, 1);
     sm100::fence_mbar_init();
     sm->abort = 0;
+    sm->exact = 0;
+    sm->qk_pend[0] = sm->qk_pend[1] = sm->v_pend = 0;
   }
   if (warp == 0) {
     sm100::tmem_alloc(&sm->tmem, TM_COLS);
     sm100::tmem_relinquish();
   }
+  if (warp == 7) load_gates(&sm->gt[0], g, beta, t0, (int)min((long long)kC, L), H, h, lane);
   sm100::tc_fence_before();
   __syncthreads();
   sm100::tc_fence_after();
   const uint32_t tmem = sm->tmem;
   const uint32_t lane_off = ((uint32_t)(warp & 3) * 32u) << 16;  // this warp's TMEM lanes
 
-  auto issue_qk = [&](long long tb) {
-    sm100::mbar_arrive_expect_tx(&sm->bar_qk, 4 * 8192);
-    sm100::tma_load_3d(gbase + OFF_STG + 0, &tm_q, &sm->bar_qk, 0, h, (int)tb);
-    sm100::tma_load_3d(gbase + OFF_STG + 8192, &tm_q, &sm->bar_qk, 64, h, (int)tb);
-    sm100::tma_load_3d(gbase + OFF_STG + 16384, &tm_k, &sm->bar_qk, 0, h, (int)tb);
-    sm100::tma_load_3d(gbase + OFF_STG + 24576, &tm_k, &sm->bar_qk, 64, h, (int)tb);
+  // TMA: chunk j's q/k into [K;Q] buffer j % 2 (K rows 0-63, Q rows 64-127 of
+  // each 64-column block, 128B-swizzled), v into the staging slot.
+  auto issue_qk = [&](long long tb, int j) {
+    const int b = j & 1;
+    uint8_t *dst = gbase + OFF_KQ + b * 32768;
+    sm100::mbar_arrive_expect_tx(&sm->bar_qk[b], 4 * 8192);
+    sm100::tma_load_3d(dst + 0, &tm_k, &sm->bar_qk[b], 0, h, (int)tb);
+    sm100::tma_load_3d(dst + 8192, &tm_q, &sm->bar_qk[b], 0, h, (int)tb);
+    sm100::tma_load_3d(dst + 16384, &tm_k, &sm->bar_qk[b], 64, h, (int)tb);
+    sm100::tma_load_3d(dst + 24576, &tm_q, &sm->bar_qk[b], 64, h, (int)tb);
+    sm->qk_pend[b] = 1 + ((j >> 1) & 1);
   };
-  auto issue_v = [&](long long tb) {
+  auto issue_v = [&](long long tb, int j) {
     sm100::mbar_arrive_expect_tx(&sm->bar_v, 2 * 8192);
-    sm100::tma_load_3d(gbase + OFF_STG + 32768, &tm_v, &sm->bar_v, 0, h, (int)tb);
-    sm100::tma_load_3d(gbase + OFF_STG + 40960, &tm_v, &sm->bar_v, 64, h, (int)tb);
+    sm100::tma_load_3d(gbase + OFF_V, &tm_v, &sm->bar_v, 0, h, (int)tb);
+    sm100::tma_load_3d(gbase + OFF_V + 8192, &tm_v, &sm->bar_v, 64, h, (int)tb);
+    sm->v_pend = 1 + (j & 1);
   };
-  // Thread 0 tracks TMA loads issued but not yet waited for, so that an
-  // aborted CTA can let them land before it exits.
-  int qk_pending = 0, v_pending = 0;  // 1 + parity of the pending phase, or 0
-  if (tid == 0) {
-    sm100::prefetch_tmap(&tm_q);
-    sm100::prefetch_tmap(&tm_k);
-    sm100::prefetch_tmap(&tm_v);
-    issue_qk(t0);
-    issue_v(t0);
-    qk_pending = v_pending = 1;
-  }
-
-  // ---- initial state: TMEM D4 (fp32) and the hi/lo fp16 operand tiles ----
-  if (tid < 128) {
-    const int k = tid;
-    for (int p = 0; p < 4; ++p) {
-      float x[32];
-#pragma unroll
-      for (int i = 0; i < 32; i += 4) {
-        float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (state_in) v4 = *reinterpret_cast<const float4 *>(state_in + st_off + k * kD + 32 * p + i);
-        x[i] = v4.x; x[i + 1] = v4.y; x[i + 2] = v4.z; x[i + 3] = v4.w;
-      }
-      sm100::tmem_st32(tmem + lane_off + TM_D4 + 32 * p, x);
-      const uint32_t blk = (uint32_t)(p >> 1) * 16384u;
-#pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        uint32_t h0, h1, h2, h3, l0, l1, l2, l3;
-        split_h2(x[8 * c4], x[8 * c4 + 1], h0, l0);
-        split_h2(x[8 * c4 + 2], x[8 * c4 + 3], h1, l1);
-        split_h2(x[8 * c4 + 4], x[8 * c4 + 5], h2, l2);
-        split_h2(x[8 * c4 + 6], x[8 * c4 + 7], h3, l3);
-        const int ch = (p & 1) * 4 + c4;
-        st_shared_v4(sw128(base + OFF_H + blk, k, ch), h0, h1, h2, h3);
-        st_shared_v4(sw128(base + OFF_H + 32768 + blk, k, ch), l0, l1, l2, l3);
-      }
-    }
-  }
-  sm100::fence_proxy_async();
-  sm100::tc_fence_before();
-  __syncthreads();
 
   const uint32_t ID_KQ = sm100::idesc_f16_f32(128, 64, 0, 0);
   const uint32_t ID_H2 = sm100::idesc_f16_f32(128, 128, 1, 0);
   const uint32_t ID_H2LO = sm100::idesc_f16_f32(128, 64, 1, 0);
   const uint32_t ID_64 = sm100::idesc_f16_f32(128, 64, 0, 0);
   const uint32_t ID_KV = sm100::idesc_f16_f32(128, 128, 1, 0);
-
-  int it = 0;
-  for (long long c0 = 0; c0 < L; c0 += kC, ++it) {
-    const int n = (int)min((long long)kC, L - c0);
-    const long long tb = t0 + c0;
-    const bool last = c0 + kC >= L;
-    const uint32_t par = (uint32_t)(it & 1);
-
-    // ---- gates of this chunk (warp 0) ----
-    if (warp == 0) {
-      float x0 = lane < n ? __ldg(g + (tb + lane) * H + h) : 0.0f;
-      float x1 = lane + 32 < n ? __ldg(g + (tb + lane + 32) * H + h) : 0.0f;
-      sm->beta[lane] = lane < n ? __ldg(beta + (tb + lane) * H + h) : 0.0f;
-      sm->beta[lane + 32] = lane + 32 < n ? __ldg(beta + (tb + lane + 32) * H + h) : 0.0f;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const float y0 = __shfl_up_sync(0xffffffffu, x0, off);
-        const float y1 = __shfl_up_sync(0xffffffffu, x1, off);
-        if (lane >= off) { x0 += y0; x1 += y1; }
-      }
-      x1 += __shfl_sync(0xffffffffu, x0, 31);
-      sm->G[lane] = x0;
-      sm->G[lane + 32] = x1;
-      __syncwarp();
-      const float gref = sm->G[(n - 1) >> 1], gn = sm->G[n - 1], g0 = sm->G[0];
-      sm->gam[lane] = expf(x0);
-      sm->gam[lane + 32] = expf(x1);
-      sm->dec[lane] = expf(gn - x0);
-      sm->dec[lane + 32] = expf(gn - x1);
-      sm->ep[lane] = expf(x0 - gref);
-      sm->ep[lane + 32] = expf(x1 - gref);
-      sm->em[lane] = expf(gref - x0);
-      sm->em[lane + 32] = expf(gref - x1);
-      if (lane == 0) {
-        sm->gn_exp = expf(gn);
-        sm->direct = (g0 - gref > 80.0f || gref - gn > 80.0f) ? 1 : 0;
-      }
-    }
-    // ---- wait for Q, K; convert to fp16 [K;Q] (rows past n zeroed) ----
-    wait_or_abort(&sm->bar_qk, par, sm, err);
-    if (tid == 0 && !sm->abort) qk_pending = 0;
-    __syncthreads();
-    if (sm->abort) break;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int e = tid + kThreads * i;  // 2048 16-byte chunks
-      const int mat = e >> 10, rem = e & 1023;
-      const int blk = rem >> 9, row = (rem >> 3) & 63, ch = rem & 7;
-      uint4 w = make_uint4(0u, 0u, 0u, 0u);
-      if (row < n) {
-        const uint4 src = ld_shared_v4(base + OFF_STG + (uint32_t)((1 - mat) * 2 + blk) * 8192u +
-                                       (uint32_t)row * 128u + (uint32_t)ch * 16u);
-        const uint32_t in[4] = {src.x, src.y, src.z, src.w};
-        uint32_t outw[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          outw[j] = pack_h2(__uint_as_float(in[j] << 16), __uint_as_float(in[j] & 0xffff0000u));
-        w = make_uint4(outw[0], outw[1], outw[2], outw[3]);
-      }
-      const int drow = mat * 64 + row;  // mat 0 = K rows 0-63, mat 1 = Q rows 64-127
-      st_shared_v4(sw128(base + OFF_KQ + (uint32_t)blk * 16384u, drow, ch), w.x, w.y, w.z, w.w);
-    }
-    sm100::fence_proxy_async();
-    __syncthreads();
-
-    // ---- MMA 1: D1 = [K;Q] K^T;  MMA 2: D2 = H0^T [K;Q]^T (hi), + H0lo^T K^T ----
-    if (tid == 0) {
-      sm100::tc_fence_after();
+  // MMAs are issued by one elected lane of a whole, converged warp (the
+  // descriptors stay warp-uniform and no sibling lane spins meanwhile).
+  auto issue_mma1 = [&](int b) {  // D1 = [K;Q] K^T
+    const uint32_t kqb = base + OFF_KQ + (uint32_t)b * 32768u;
+    if (sm100::elect_one()) {
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
-        const uint32_t a = base + OFF_KQ + (uint32_t)(ks >> 2) * 16384u + (uint32_t)(ks & 3) * 32u;
+        const uint32_t a = kqb + (uint32_t)(ks >> 2) * 16384u + (uint32_t)(ks & 3) * 32u;
         sm100::mma_f16_ss(tmem + TM_D1, kdesc(a), kdesc(a), ID_KQ, ks > 0);
       }
       sm100::mma_commit(&sm->bar_m1);
+    }
+    __syncwarp();
+  };
+
+  const int n_chunks = (int)((L + kC - 1) / kC);
+  if (tid == 0) {
+    sm100::prefetch_tmap(&tm_q);
+    sm100::prefetch_tmap(&tm_k);
+    sm100::prefetch_tmap(&tm_v);
+    issue_qk(t0, 0);
+    issue_v(t0, 0);
+    if (n_chunks > 1) issue_qk(t0 + kC, 1);
+  }
+
+  // ---- initial state: TMEM D4 = gamma_n * H0 (fp32) and H0 hi/lo tiles;
+  //      each warp: 32 key rows x 64 value columns (warpgroup half) ----
+  {
+    const float gnx = sm->gt[0].gn_exp;
+#pragma unroll 1
+    for (int p = 0; p < 2; ++p) {
+      const int c0 = 64 * wg + 32 * p;
+      float x[32];
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        const uint32_t b = base + OFF_KQ + (uint32_t)(ks >> 2) * 16384u + (uint32_t)(ks & 3) * 32u;
-        sm100::mma_f16_ss(tmem + TM_D2, mndesc(base + OFF_H + (uint32_t)ks * 2048u, 16384),
-                          kdesc(b), ID_H2, ks > 0);
+      for (int i = 0; i < 32; i += 4) {
+        float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (state_in) v4 = *reinterpret_cast<const float4 *>(state_in + st_off + row * kD + c0 + i);
+        x[i] = v4.x; x[i + 1] = v4.y; x[i + 2] = v4.z; x[i + 3] = v4.w;
       }
+      store32_hl(base + OFF_H + 16384u * wg, base + OFF_H + 32768u + 16384u * wg, row, 4 * p, x);
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        const uint32_t b = base + OFF_KQ + (uint32_t)(ks >> 2) * 16384u + (uint32_t)(ks & 3) * 32u;
-        sm100::mma_f16_ss(tmem + TM_D2, mndesc(base + OFF_H + 32768u + (uint32_t)ks * 2048u, 16384),
-                          kdesc(b), ID_H2LO, 1);
+      for (int i = 0; i < 32; ++i) x[i] *= gnx;
+      sm100::tmem_st32(tmem + lane_off + TM_D4 + c0, x);
+    }
+  }
+  // ---- chunk 0's [K;Q]: wait, convert, MMA1 (later chunks' are prepared
+  //      during the previous chunk) ----
+  if (wait_or_abort(&sm->bar_qk[0], 0, sm, err) && tid == 0) sm->qk_pend[0] = 0;
+  convert_kq(base + OFF_KQ, (int)min((long long)kC, L), tid, kThreads);
+  sm100::fence_proxy_async();
+  sm100::tc_fence_before();
+  __syncthreads();
+  if (warp == 0 && !sm->abort) {
+    sm100::tc_fence_after();
+    issue_mma1(0);
+  }
+
+  int it = 0;
+  for (long long c0 = 0; c0 < L && !sm->abort; c0 += kC, ++it) {
+    const int n = (int)min((long long)kC, L - c0);
+    const long long tb = t0 + c0;
+    const bool last = it == n_chunks - 1;
+    const uint32_t par = (uint32_t)(it & 1);
+    const int kb = it & 1;
+    const uint32_t kq = base + OFF_KQ + (uint32_t)kb * 32768u;
+    const Gates *gt = &sm->gt[it & 1];
+    Gates *gt_next = &sm->gt[(it + 1) & 1];
+    const bool exact = sm->exact != 0;
+    // H0's FP8 tile scale for this thread's value row (read before epilogue 4
+    // overwrites it with the next chunk's scales)
+    const float hsv = exact ? sm->hs[row >> 6] : 1.0f;
+
+    // ---- MMA 2: D2 = H0^T [K;Q]^T (hi, or exact codes), + H0lo^T K^T ----
+    if (warp == 0) {
+      sm100::tc_fence_after();
+      if (sm100::elect_one()) {
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t b = kq + (uint32_t)(ks >> 2) * 16384u + (uint32_t)(ks & 3) * 32u;
+          sm100::mma_f16_ss(tmem + TM_D2, mndesc(base + OFF_H + (uint32_t)ks * 2048u, 16384),
+                            kdesc(b), ID_H2, ks > 0);
+        }
+        if (!exact) {
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint32_t b = kq + (uint32_t)(ks >> 2) * 16384u + (uint32_t)(ks & 3) * 32u;
+            sm100::mma_f16_ss(tmem + TM_D2,
+                              mndesc(base + OFF_H + 32768u + (uint32_t)ks * 2048u, 16384),
+                              kdesc(b), ID_H2LO, 1);
+          }
+        }
+        sm100::mma_commit(&sm->bar_m2);
       }
-      sm100::mma_commit(&sm->bar_m2);
+      __syncwarp();
     }
 
-    // ---- epilogue 1: A (fp32, for the solve) and Aqk (fp16 operand) ----
-    if (tid < 128) {
+    // ---- epilogue 1 (all warps; warps w and w + 4 split D1's 64 columns):
+    //      rows 0-63 -> A (fp32, for the solve), rows 64-127 -> Aqk (fp16) ----
+    {
       wait_or_abort(&sm->bar_m1, par, sm, err);
       sm100::tc_fence_after();
-      float v[64];
-      sm100::tmem_ld32(tmem + lane_off + TM_D1, *reinterpret_cast<float(*)[32]>(v));
-      sm100::tmem_ld32(tmem + lane_off + TM_D1 + 32, *reinterpret_cast<float(*)[32]>(v + 32));
-      const bool direct = sm->direct != 0;
-      if (tid < 64) {
-        const int r = tid;
-        const float br = sm->beta[r], epr = sm->ep[r], Gr = sm->G[r];
+      const int r = row & 63, i0 = 32 * wg;
+      float v[32];
+      sm100::tmem_ld32(tmem + lane_off + TM_D1 + i0, v);
+      if (gt->direct) {
+        const float Gr = gt->G[r];
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          const float e = direct ? expf(Gr - sm->G[i]) : epr * sm->em[i];
-          sA[r * LDS + i] = i < r ? br * e * v[i] : 0.0f;
-        }
+        for (int i = 0; i < 32; ++i) v[i] *= expf(Gr - gt->G[i0 + i]);
       } else {
-        const int r = tid - 64;
-        const float epr = sm->ep[r], Gr = sm->G[r];
+        const float epr = gt->ep[r];
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          const float e = direct ? expf(Gr - sm->G[i]) : epr * sm->em[i];
-          v[i] = i <= r ? e * v[i] : 0.0f;
+        for (int i = 0; i < 32; i += 4) {
+          const float4 e4 = *reinterpret_cast<const float4 *>(gt->em + i0 + i);
+          v[i] *= epr * e4.x; v[i + 1] *= epr * e4.y; v[i + 2] *= epr * e4.z; v[i + 3] *= epr * e4.w;
         }
-        store_row_h(base + OFF_AQK, r, v);
+      }
+      if (row < 64) {
+        const float br = gt->beta[r];
+        float *arow = sA + r * LDT + i0;
+#pragma unroll
+        for (int i = 0; i < 32; i += 4)
+          *reinterpret_cast<float4 *>(arow + i) =
+              make_float4(i0 + i < r ? br * v[i] : 0.f, i0 + i + 1 < r ? br * v[i + 1] : 0.f,
+                          i0 + i + 2 < r ? br * v[i + 2] : 0.f, i0 + i + 3 < r ? br * v[i + 3] : 0.f);
+      } else {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float y[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) y[e] = i0 + 8 * c + e <= r ? v[8 * c + e] : 0.f;
+          st_shared_v4(sw128(base + OFF_AQK, r, 4 * wg + c), pack_h2(y[0], y[1]),
+                       pack_h2(y[2], y[3]), pack_h2(y[4], y[5]), pack_h2(y[6], y[7]));
+        }
       }
     }
     sm100::fence_proxy_async();
     __syncthreads();
     if (sm->abort) break;
 
-    // ---- triangular solve T = (I + A)^-1, blocked by 16 ----
-    // Diagonal blocks: column substitution, one thread per column.
-    if (tid < 64) {
-      const int b = tid >> 4, jj = tid & 15, j0 = 16 * b;
-      float x[16];
+    if (wg == 0) {
+      // ---- WG0: triangular solve T = (I + A)^-1 in three levels ----
+      // Level 0: the 16x16 diagonal blocks by column substitution (warps 0-1,
+      // one thread per column); warps 2-3 zero the blocks (0,1) and (2,3)
+      // above the diagonal that the 32x32 level reads.
+      if (tid < 64) {
+        // right-looking: once x[m] is final it updates every later row, so
+        // the dependent chain is 16 steps long instead of 120
+        const int b = tid >> 4, jj = tid & 15, j0 = 16 * b;
+        const float *ablk = sA + j0 * LDT + j0;
+        float x[16];
 #pragma unroll
-      for (int rr = 0; rr < 16; ++rr) {
-        float acc = rr == jj ? 1.0f : 0.0f;
-        if (rr > jj) {
+        for (int rr = 0; rr < 16; ++rr) x[rr] = rr == jj ? 1.0f : 0.0f;
 #pragma unroll
-          for (int m = 0; m < rr; ++m) acc -= sA[(j0 + rr) * LDS + j0 + m] * x[m];
+        for (int m = 0; m < 15; ++m) {
+#pragma unroll
+          for (int rr = m + 1; rr < 16; ++rr) x[rr] -= ablk[rr * LDT + m] * x[m];
         }
-        x[rr] = acc;
-      }
+        float *tcol = sT + j0 * LDT + j0 + jj;
 #pragma unroll
-      for (int rr = 0; rr < 16; ++rr) sT[(j0 + rr) * LDS + j0 + jj] = x[rr];
-    }
-    __syncthreads();
-    // Block rows 1..3: P = A[rows, :] T[:, cols] over the solved part, then
-    // T[rows, cols] = -T_ii P.
-    for (int bi = 1; bi < 4; ++bi) {
-      const int r0 = 16 * bi, ncol = 16 * bi, nel = 16 * ncol;
-      for (int e = tid; e < nel; e += kThreads) {
-        const int rr = e / ncol, c = e % ncol;
-        float acc = 0.0f;
-        for (int m = c; m < r0; ++m) acc += sA[(r0 + rr) * LDS + m] * sT[m * LDS + c];
-        sP[rr * LDS + c] = acc;
-      }
-      __syncthreads();
-      for (int e = tid; e < nel; e += kThreads) {
-        const int rr = e / ncol, c = e % ncol;
-        float acc = 0.0f;
-        for (int m = 0; m <= rr; ++m) acc += sT[(r0 + rr) * LDS + r0 + m] * sP[m * LDS + c];
-        sT[(r0 + rr) * LDS + c] = -acc;
-      }
-      __syncthreads();
-    }
-    // T -> hi/lo fp16 tiles [tok][tok'] (upper triangle zero).
-    {
-      const int r = tid >> 2, cpart = (tid & 3) * 16;
-      float x[16];
+        for (int rr = 0; rr < 16; ++rr) tcol[rr * LDT] = x[rr];
+      } else {
+        const int e = tid - 64;  // 64 threads x 8 values
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int c = cpart + i;
-        x[i] = c <= r ? sT[r * LDS + c] : 0.0f;
+        for (int i = 0; i < 8; ++i) {
+          const int idx = e * 8 + i, b = idx >> 8, rr = (idx >> 4) & 15, cc = idx & 15;
+          sT[(32 * b + rr) * LDT + 32 * b + 16 + cc] = 0.0f;
+        }
       }
+      asm volatile("bar.sync 3, 128;" ::: "memory");
+      // Level 1: blocks (1,0) and (3,2): T_ij = -T_ii (A_ij T_jj).
+      {
+        const int blk = tid >> 6, idx = tid & 63, rr = idx >> 2, cc = (idx & 3) * 4;
+        const int r0 = 16 + 32 * blk, c0b = 32 * blk;
+        const float *arow = sA + (r0 + rr) * LDT + c0b;
+        const float *tcol = sT + c0b * LDT + c0b + cc;
+        float4 p = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t h0, h1, h2, h3, l0, l1, l2, l3;
-        const float *y = x + 8 * half;
-        split_h2(y[0], y[1], h0, l0);
-        split_h2(y[2], y[3], h1, l1);
-        split_h2(y[4], y[5], h2, l2);
-        split_h2(y[6], y[7], h3, l3);
-        const int ch = (cpart >> 3) + half;
-        st_shared_v4(sw128(base + OFF_X + X_THI, r, ch), h0, h1, h2, h3);
-        st_shared_v4(sw128(base + OFF_X + X_TLO, r, ch), l0, l1, l2, l3);
+        for (int m = 0; m < 16; ++m) {
+          const float a = arow[m];
+          const float4 t4 = *reinterpret_cast<const float4 *>(tcol + m * LDT);
+          p.x += a * t4.x; p.y += a * t4.y; p.z += a * t4.z; p.w += a * t4.w;
+        }
+        *reinterpret_cast<float4 *>(sP + (16 * blk + rr) * LDT + cc) = p;
+        asm volatile("bar.sync 3, 128;" ::: "memory");
+        const float *trow = sT + (r0 + rr) * LDT + r0;
+        const float *pcol = sP + 16 * blk * LDT + cc;
+        float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int m = 0; m < 16; ++m) {
+          const float t = trow[m];
+          const float4 p4 = *reinterpret_cast<const float4 *>(pcol + m * LDT);
+          q.x += t * p4.x; q.y += t * p4.y; q.z += t * p4.z; q.w += t * p4.w;
+        }
+        *reinterpret_cast<float4 *>(sT + (r0 + rr) * LDT + c0b + cc) =
+            make_float4(-q.x, -q.y, -q.z, -q.w);
       }
-    }
-    sm100::fence_proxy_async();
-    __syncthreads();
-    // staging Q/K (which held the solve's fp32 T) is free: prefetch the next chunk
-    if (tid == 0 && !last) {
-      issue_qk(tb + kC);
-      qk_pending = 1 + ((it + 1) & 1);
-    }
-
-    // ---- epilogue 2: R = diag(beta) (V - diag(gamma) P) -> R^T hi/lo;
-    //      O accumulator initialised with gamma-scaled (Q H0)^T ----
-    wait_or_abort(&sm->bar_v, par, sm, err);
-    if (tid == 0 && !sm->abort) v_pending = 0;
-    if (tid < 128) {
+      asm volatile("bar.sync 3, 128;" ::: "memory");
+      // Level 2: the lower-left 32x32 block: T_21 = -T_22 (A_21 T_11).
+      {
+        const int rr = tid >> 2, cc = (tid & 3) * 8;
+        const float *arow = sA + (32 + rr) * LDT;
+        const float *tcol = sT + cc;
+        float p[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int m = 0; m < 32; ++m) {
+          const float a = arow[m];
+          const float4 t0v = *reinterpret_cast<const float4 *>(tcol + m * LDT);
+          const float4 t1v = *reinterpret_cast<const float4 *>(tcol + m * LDT + 4);
+          p[0] += a * t0v.x; p[1] += a * t0v.y; p[2] += a * t0v.z; p[3] += a * t0v.w;
+          p[4] += a * t1v.x; p[5] += a * t1v.y; p[6] += a * t1v.z; p[7] += a * t1v.w;
+        }
+        *reinterpret_cast<float4 *>(sP + rr * LDT + cc) = make_float4(p[0], p[1], p[2], p[3]);
+        *reinterpret_cast<float4 *>(sP + rr * LDT + cc + 4) = make_float4(p[4], p[5], p[6], p[7]);
+        asm volatile("bar.sync 3, 128;" ::: "memory");
+        const float *trow = sT + (32 + rr) * LDT + 32;
+        const float *pcol = sP + cc;
+        float q[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int m = 0; m < 32; ++m) {
+          const float t = trow[m];
+          const float4 p0v = *reinterpret_cast<const float4 *>(pcol + m * LDT);
+          const float4 p1v = *reinterpret_cast<const float4 *>(pcol + m * LDT + 4);
+          q[0] += t * p0v.x; q[1] += t * p0v.y; q[2] += t * p0v.z; q[3] += t * p0v.w;
+          q[4] += t * p1v.x; q[5] += t * p1v.y; q[6] += t * p1v.z; q[7] += t * p1v.w;
+        }
+        float *tout = sT + (32 + rr) * LDT + cc;
+        *reinterpret_cast<float4 *>(tout) = make_float4(-q[0], -q[1], -q[2], -q[3]);
+        *reinterpret_cast<float4 *>(tout + 4) = make_float4(-q[4], -q[5], -q[6], -q[7]);
+      }
+      asm volatile("bar.sync 3, 128;" ::: "memory");
+      // T -> hi/lo fp16 tiles [tok][tok'] (upper triangle zero).
+      {
+        const int r = tid >> 1, cpart = (tid & 1) * 32;
+        const float *trow = sT + r * LDT + cpart;
+        float x[32];
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) {
+          const float4 t4 = *reinterpret_cast<const float4 *>(trow + i);
+          x[i] = cpart + i <= r ? t4.x : 0.f;
+          x[i + 1] = cpart + i + 1 <= r ? t4.y : 0.f;
+          x[i + 2] = cpart + i + 2 <= r ? t4.z : 0.f;
+          x[i + 3] = cpart + i + 3 <= r ? t4.w : 0.f;
+        }
+        store32_hl(base + OFF_X + X_THI, base + OFF_X + X_TLO, r, cpart >> 3, x);
+      }
+    } else {
+      // ---- WG1, epilogue 2: R = diag(beta) (V - diag(gamma) P) -> TMEM as
+      //      the A operand of MMA 3; then the next chunk's gates (warp 7) ----
+      if (wait_or_abort(&sm->bar_v, par, sm, err) && tid == 128) sm->v_pend = 0;
       wait_or_abort(&sm->bar_m2, par, sm, err);
       sm100::tc_fence_after();
-      const int vv = tid;
-      const uint8_t *stgv = gbase + OFF_STG + 32768 + (vv >> 6) * 8192 + (vv & 63) * 2;
-      float x[64];
-      sm100::tmem_ld32(tmem + lane_off + TM_D2, *reinterpret_cast<float(*)[32]>(x));
-      sm100::tmem_ld32(tmem + lane_off + TM_D2 + 32, *reinterpret_cast<float(*)[32]>(x + 32));
-#pragma unroll
-      for (int t = 0; t < 64; ++t) {
-        const float vt = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(stgv + t * 128));
-        x[t] = t < n ? sm->beta[t] * (vt - sm->gam[t] * x[t]) : 0.0f;
+      if (n < kC) {  // a partial last chunk: rows past n read as zero
+        for (int e = tid - 128; e < 2 * 64 * 8; e += 128) {
+          const int blk = e >> 9, rw = (e >> 3) & 63, ch = e & 7;
+          if (rw >= n) st_shared_v4(base + OFF_V + blk * 8192 + rw * 128 + ch * 16, 0u, 0u, 0u, 0u);
+        }
+        asm volatile("bar.sync 4, 128;" ::: "memory");
       }
-      store_row_hl(base + OFF_X + X_RHI, base + OFF_X + X_RLO, vv, x);
+      const uint8_t *stgv = gbase + OFF_V + (row >> 6) * 8192 + (row & 63) * 2;
 #pragma unroll
-      for (int p = 0; p < 2; ++p) {
-        float y[32];
-        sm100::tmem_ld32(tmem + lane_off + TM_D2 + 64 + 32 * p, y);
+      for (int half = 0; half < 2; ++half) {
+        float x[32];
+        sm100::tmem_ld32(tmem + lane_off + TM_D2 + 32 * half, x);
+        uint32_t whi[16], wlo[16];
 #pragma unroll
-        for (int t = 0; t < 32; ++t) y[t] *= sm->gam[32 * p + t];
-        sm100::tmem_st32(tmem + lane_off + TM_D2 + 64 + 32 * p, y);
+        for (int t = 0; t < 32; t += 4) {
+          const int tok = 32 * half + t;
+          const float4 b4 = *reinterpret_cast<const float4 *>(gt->beta + tok);
+          const float4 g4 = *reinterpret_cast<const float4 *>(gt->gam + tok);
+          const float bb[4] = {b4.x, b4.y, b4.z, b4.w}, gg[4] = {g4.x, g4.y, g4.z, g4.w};
+          float r4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float vt =
+                __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(stgv + (tok + e) * 128));
+            // past n: beta, v and P (K rows zeroed) are all zero, so R is 0
+            r4[e] = bb[e] * (vt - (gg[e] * hsv) * x[t + e]);
+          }
+          split_h2(r4[0], r4[1], whi[t >> 1], wlo[t >> 1]);
+          split_h2(r4[2], r4[3], whi[(t >> 1) + 1], wlo[(t >> 1) + 1]);
+        }
+        sm100::tmem_st16(tmem + lane_off + TM_RHI + 16 * half, whi);
+        sm100::tmem_st16(tmem + lane_off + TM_RLO + 16 * half, wlo);
       }
-    }
-    sm100::fence_proxy_async();
-    sm100::tc_fence_before();
-    __syncthreads();
-    if (sm->abort) break;
-    if (tid == 0 && !last) {
-      issue_v(tb + kC);
-      v_pending = 1 + ((it + 1) & 1);
-    }
-
-    // ---- MMA 3: Vn^T = R^T T^T (hi*hi + hi*lo + lo*hi) ----
-    if (tid == 0) {
-      sm100::tc_fence_after();
-      const uint32_t rA[3] = {X_RHI, X_RHI, X_RLO}, tB[3] = {X_THI, X_TLO, X_THI};
-#pragma unroll
-      for (int pass = 0; pass < 3; ++pass)
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          sm100::mma_f16_ss(tmem + TM_D3, kdesc(base + OFF_X + rA[pass] + 32u * ks),
-                            kdesc(base + OFF_X + tB[pass] + 32u * ks), ID_64, pass + ks > 0);
-      sm100::mma_commit(&sm->bar_m3);
-    }
-
-    // ---- epilogue 3: Vn^T hi and decayed dVn^T hi/lo; H accumulator *= gamma_n ----
-    if (tid < 128) {
-      wait_or_abort(&sm->bar_m3, par, sm, err);
-      sm100::tc_fence_after();
-      const int vv = tid;
-      float x[64];
-      sm100::tmem_ld32(tmem + lane_off + TM_D3, *reinterpret_cast<float(*)[32]>(x));
-      sm100::tmem_ld32(tmem + lane_off + TM_D3 + 32, *reinterpret_cast<float(*)[32]>(x + 32));
-      store_row_h(base + OFF_X + X_VN, vv, x);
-#pragma unroll
-      for (int t = 0; t < 64; ++t) x[t] *= sm->dec[t];
-      store_row_hl(base + OFF_X + X_DVHI, base + OFF_X + X_DVLO, vv, x);
-      const float gnx = sm->gn_exp;
-#pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        float y[32];
-        sm100::tmem_ld32(tmem + lane_off + TM_D4 + 32 * p, y);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) y[i] *= gnx;
-        sm100::tmem_st32(tmem + lane_off + TM_D4 + 32 * p, y);
-      }
-    }
-    sm100::fence_proxy_async();
-    sm100::tc_fence_before();
-    __syncthreads();
-    if (sm->abort) break;
-
-    // ---- MMA 4: O^T += Vn^T Aqk^T;  MMA 5: H += K^T dVn (hi, lo) ----
-    if (tid == 0) {
-      sm100::tc_fence_after();
-#pragma unroll
-      for (int ks = 0; ks < 4; ++ks)
-        sm100::mma_f16_ss(tmem + TM_D2 + 64, kdesc(base + OFF_X + X_VN + 32u * ks),
-                          kdesc(base + OFF_AQK + 32u * ks), ID_64, 1);
-#pragma unroll
-      for (int pass = 0; pass < 2; ++pass)
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          sm100::mma_f16_ss(tmem + TM_D4, mndesc(base + OFF_KQ + (uint32_t)ks * 2048u, 16384),
-                            kdesc(base + OFF_X + (pass ? X_DVLO : X_DVHI) + 32u * ks), ID_KV, 1);
-      sm100::mma_commit(&sm->bar_m4);
-    }
-
-    // ---- epilogue 4: outputs, state QDQ, next chunk's H0 operands ----
-    if (tid < 128) {
-      wait_or_abort(&sm->bar_m4, par, sm, err);
-      sm100::tc_fence_after();
-      // O^T[v][t] -> o[t][h][v]
-      const int vv = tid;
-#pragma unroll
-      for (int p = 0; p < 2; ++p) {
-        float y[32];
-        sm100::tmem_ld32(tmem + lane_off + TM_D2 + 64 + 32 * p, y);
-#pragma unroll
-        for (int t = 0; t < 32; ++t) {
-          const int tok = 32 * p + t;
-          if (tok < n) o[((tb + tok) * H + h) * kD + vv] = __float2bfloat16_rn(scale * y[t]);
+      if (warp == 7 && !last)
+        load_gates(gt_next, g, beta, tb + kC, (int)min((long long)kC, L - c0 - kC), H, h, lane);
+      if (!last) {
+        // Still inside WG0's solve: prepare the next chunk - convert its
+        // [K;Q] (landed by TMA a chunk ago) and issue its MMA 1 (D1 was read
+        // by epilogue 1 already).
+        const int nb = kb ^ 1;
+        if (wait_or_abort(&sm->bar_qk[nb], (uint32_t)(((it + 1) >> 1) & 1), sm, err) && tid == 128)
+          sm->qk_pend[nb] = 0;
+        convert_kq(base + OFF_KQ + (uint32_t)nb * 32768u, (int)min((long long)kC, L - c0 - kC),
+                   tid - 128, 128);
+        sm100::fence_proxy_async();
+        asm volatile("bar.sync 4, 128;" ::: "memory");
+        if (warp == 4 && !sm->abort) {
+          sm100::tc_fence_after();
+          issue_mma1(nb);
         }
       }
-      // H rows: this thread owns key row k = tid.  Pass 1 (FP8 tiles, INT8
-      // groups of 64): amax of the two 64-column halves of the row; FP8 then
-      // reduces them over all 128 rows (the tile spans every key).
-      const int k = tid;
-      float mh[2] = {0.f, 0.f};
+    }
+    sm100::fence_proxy_async();
+    sm100::tc_fence_before();
+    __syncthreads();
+    if (sm->abort) break;
+    if (tid == 0 && !last) issue_v(tb + kC, it + 1);
+
+    // ---- MMA 3: Vn^T = R^T T^T (hi*hi + hi*lo + lo*hi), R^T from TMEM ----
+    if (warp == 0) {
+      sm100::tc_fence_after();
+      if (sm100::elect_one()) {
+        const uint32_t rA[3] = {TM_RHI, TM_RHI, TM_RLO}, tB[3] = {X_THI, X_TLO, X_THI};
+#pragma unroll
+        for (int pass = 0; pass < 3; ++pass)
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            sm100::mma_f16_ts(tmem + TM_D3, tmem + rA[pass] + 8u * ks,
+                              kdesc(base + OFF_X + tB[pass] + 32u * ks), ID_64, pass + ks > 0);
+        sm100::mma_commit(&sm->bar_m3);
+      }
+      __syncwarp();
+    }
+
+    // ---- epilogue 3: Vn^T hi -> TMEM (A of MMA 4); decayed dVn^T hi/lo -> smem ----
+    {
+      wait_or_abort(&sm->bar_m3, par, sm, err);
+      sm100::tc_fence_after();
+      const int vv = row, t0h = 32 * wg;
+      float x[32];
+      sm100::tmem_ld32(tmem + lane_off + TM_D3 + t0h, x);
+      uint32_t w[16];
+#pragma unroll
+      for (int t = 0; t < 32; t += 2) w[t >> 1] = pack_h2(x[t], x[t + 1]);
+      sm100::tmem_st16(tmem + lane_off + TM_VN + 16 * wg, w);
+#pragma unroll
+      for (int t = 0; t < 32; ++t) x[t] *= gt->dec[t0h + t];
+      store32_hl(base + OFF_X + X_DVHI, base + OFF_X + X_DVLO, vv, 4 * wg, x);
+    }
+    sm100::fence_proxy_async();
+    sm100::tc_fence_before();
+    __syncthreads();
+    if (sm->abort) break;
+
+    // ---- MMA 4: D5 = Vn^T Aqk^T (Vn^T from TMEM);  MMA 5: H += K^T dVn ----
+    if (warp == 0) {
+      sm100::tc_fence_after();
+      if (sm100::elect_one()) {
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          sm100::mma_f16_ts(tmem + TM_D5, tmem + TM_VN + 8u * ks,
+                            kdesc(base + OFF_AQK + 32u * ks), ID_64, ks > 0);
+#pragma unroll
+        for (int pass = 0; pass < 2; ++pass)
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            sm100::mma_f16_ss(tmem + TM_D4, mndesc(kq + (uint32_t)ks * 2048u, 16384),
+                              kdesc(base + OFF_X + (pass ? X_DVLO : X_DVHI) + 32u * ks), ID_KV, 1);
+        sm100::mma_commit(&sm->bar_m4);
+      }
+      __syncwarp();
+    }
+
+    // ---- epilogue 4 ----
+    wait_or_abort(&sm->bar_m4, par, sm, err);
+    sm100::tc_fence_after();
+    // the buffer MMA 5 just released takes the chunk after next
+    if (tid == 128 && !last && it + 2 < n_chunks && !sm->abort) issue_qk(tb + 2 * kC, it + 2);
+    {
+      // O^T[v][t] = scale (gamma_t (Q H0)^T[v][t] + (Aqk Vn)^T[v][t]) ->
+      // o[t][h][v]: warpgroup wg writes tokens 32 wg .. + 31
+      {
+        float qh[32], av[32];
+        sm100::tmem_ld32(tmem + lane_off + TM_D2 + 64 + 32 * wg, qh);
+        sm100::tmem_ld32(tmem + lane_off + TM_D5 + 32 * wg, av);
+        __nv_bfloat16 *op = o + ((tb + 32 * wg) * H + h) * kD + row;
+        const long long ts = (long long)H * kD;
+        const float sh = scale * hsv;
+#pragma unroll
+        for (int t = 0; t < 32; t += 4) {
+          const float4 g4 = *reinterpret_cast<const float4 *>(gt->gam + 32 * wg + t);
+          qh[t] = fmaf(sh * g4.x, qh[t], scale * av[t]);
+          qh[t + 1] = fmaf(sh * g4.y, qh[t + 1], scale * av[t + 1]);
+          qh[t + 2] = fmaf(sh * g4.z, qh[t + 2], scale * av[t + 2]);
+          qh[t + 3] = fmaf(sh * g4.w, qh[t + 3], scale * av[t + 3]);
+        }
+        if (n == kC) {
+#pragma unroll
+          for (int t = 0; t < 32; ++t) op[t * ts] = __float2bfloat16_rn(qh[t]);
+        } else {
+#pragma unroll
+          for (int t = 0; t < 32; ++t)
+            if (32 * wg + t < n) op[t * ts] = __float2bfloat16_rn(qh[t]);
+        }
+      }
+      // H: key row `row`, value columns 64 wg .. + 63 (one FP8 tile per
+      // warpgroup).  Pass 1 (FP8 tiles, INT8 groups of 64): amax of the 64
+      // columns, for FP8 reduced over the warpgroup's 128 rows.
+      float mh = 0.f;
       if (QK == kQdqFp8Tile || (QK == kQdqInt8 && GROUP == 64)) {
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
+        for (int p = 0; p < 2; ++p) {
           float y[32];
-          sm100::tmem_ld32(tmem + lane_off + TM_D4 + 32 * p, y);
-          float m = 0.f;
+          sm100::tmem_ld32(tmem + lane_off + TM_D4 + 64 * wg + 32 * p, y);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(y[i]));
-          mh[p >> 1] = fmaxf(mh[p >> 1], m);
+          for (int i = 0; i < 32; ++i) mh = fmaxf(mh, fabsf(y[i]));
         }
       }
       if (QK == kQdqFp8Tile) {
-        const float m0 = group_max<32>(mh[0]), m1 = group_max<32>(mh[1]);
-        if (lane == 0) { sm->red[2 * warp] = m0; sm->red[2 * warp + 1] = m1; }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        mh[0] = fmaxf(fmaxf(sm->red[0], sm->red[2]), fmaxf(sm->red[4], sm->red[6]));
-        mh[1] = fmaxf(fmaxf(sm->red[1], sm->red[3]), fmaxf(sm->red[5], sm->red[7]));
-        asm volatile("bar.sync 1, 128;" ::: "memory");
+        mh = group_max<32>(mh);
+        if (lane == 0) sm->red[wg][warp & 3] = mh;
+        asm volatile("bar.sync %0, 128;" ::"r"(1 + wg) : "memory");
+        mh = fmaxf(fmaxf(sm->red[wg][0], sm->red[wg][1]), fmaxf(sm->red[wg][2], sm->red[wg][3]));
       }
-      // Pass 2: quantize, write back the fp32 state, its hi/lo operand tiles
-      // and, after the last chunk, state_out.
+      const float gn_next = last ? 1.0f : sm->gt[(it + 1) & 1].gn_exp;
+      const ScaleRecip sr_tile = make_scale(fp8_scale(QK == kQdqFp8Tile && mh > 0.f ? mh : 1.0f));
+      // Pass 2: quantize; H0 operand tiles (exact codes for FP8, hi/lo
+      // otherwise); gamma_n(next) * H into TMEM as the next carry's
+      // accumulator; state_out after the last chunk.
 #pragma unroll
-      for (int p = 0; p < 4; ++p) {
+      for (int p = 0; p < 2; ++p) {
+        const int c0v = 64 * wg + 32 * p;
         float y[32];
-        sm100::tmem_ld32(tmem + lane_off + TM_D4 + 32 * p, y);
-        if (QK == kQdqInt8) {
-          constexpr int GW = GROUP < 32 ? GROUP : 32;  // group width inside this piece
-#pragma unroll
-          for (int g0 = 0; g0 < 32; g0 += GW) {
-            float m = 0.f;
-            if (GROUP == 64) {
-              m = mh[p >> 1];
-            } else {
-#pragma unroll
-              for (int i = 0; i < GW; ++i) m = fmaxf(m, fabsf(y[g0 + i]));
-            }
-            if (m == 0.0f) {
-#pragma unroll
-              for (int i = 0; i < GW; ++i) y[g0 + i] = 0.0f;
-            } else {
-              const ScaleRecip sr = make_scale(int8_scale(m));
-#pragma unroll
-              for (int i = 0; i < GW; ++i) y[g0 + i] = qdq_int8(y[g0 + i], sr);
-            }
-          }
-          sm100::tmem_st32(tmem + lane_off + TM_D4 + 32 * p, y);
-        } else if (QK == kQdqFp8Tile) {
-          const float m = mh[p >> 1];
-          if (m == 0.0f) {
+        sm100::tmem_ld32(tmem + lane_off + TM_D4 + c0v, y);
+        if (QK == kQdqFp8Tile) {
+          uint32_t code[16];
+          if (mh == 0.0f) {  // zero tile: codes and values 0
 #pragma unroll
             for (int i = 0; i < 32; ++i) y[i] = 0.0f;
-          } else {
-            const ScaleRecip sr = make_scale(fp8_scale(m));
 #pragma unroll
-            for (int i = 0; i < 32; i += 2) {
-              const float2 r2 = qdq_fp8_2(y[i], y[i + 1], sr);
-              y[i] = r2.x;
-              y[i + 1] = r2.y;
+            for (int i = 0; i < 16; ++i) code[i] = 0u;
+          } else if (sr_tile.pre == 1.0f) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 2)
+              code[i >> 1] = fp8_code_pair(y[i], y[i + 1], sr_tile.s, sr_tile.r, y[i], y[i + 1]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; i += 2)
+              code[i >> 1] = fp8_code_pair(y[i] * sr_tile.pre, y[i + 1] * sr_tile.pre, sr_tile.s2,
+                                           sr_tile.r, y[i], y[i + 1], sr_tile.s);
+          }
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            st_shared_v4(sw128(base + OFF_H + 16384u * wg, row, 4 * p + c), code[4 * c],
+                         code[4 * c + 1], code[4 * c + 2], code[4 * c + 3]);
+        } else {
+          if (QK == kQdqInt8) {
+            constexpr int GW = GROUP < 32 ? GROUP : 32;  // group width inside this piece
+#pragma unroll
+            for (int g0 = 0; g0 < 32; g0 += GW) {
+              float m = 0.f;
+              if (GROUP == 64) {
+                m = mh;
+              } else {
+#pragma unroll
+                for (int i = 0; i < GW; ++i) m = fmaxf(m, fabsf(y[g0 + i]));
+              }
+              if (m == 0.0f) {
+#pragma unroll
+                for (int i = 0; i < GW; ++i) y[g0 + i] = 0.0f;
+              } else {
+                const ScaleRecip sr = make_scale(int8_scale(m));
+#pragma unroll
+                for (int i = 0; i < GW; ++i) y[g0 + i] = qdq_int8(y[g0 + i], sr);
+              }
             }
           }
-          sm100::tmem_st32(tmem + lane_off + TM_D4 + 32 * p, y);
-        }
-        const uint32_t blk = (uint32_t)(p >> 1) * 16384u;
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          uint32_t h0, h1, h2, h3, l0, l1, l2, l3;
-          split_h2(y[8 * c4], y[8 * c4 + 1], h0, l0);
-          split_h2(y[8 * c4 + 2], y[8 * c4 + 3], h1, l1);
-          split_h2(y[8 * c4 + 4], y[8 * c4 + 5], h2, l2);
-          split_h2(y[8 * c4 + 6], y[8 * c4 + 7], h3, l3);
-          const int ch = (p & 1) * 4 + c4;
-          st_shared_v4(sw128(base + OFF_H + blk, k, ch), h0, h1, h2, h3);
-          st_shared_v4(sw128(base + OFF_H + 32768 + blk, k, ch), l0, l1, l2, l3);
+          store32_hl(base + OFF_H + 16384u * wg, base + OFF_H + 32768u + 16384u * wg, row,
+                     4 * p, y);
         }
         if (last) {
-          float *dst = state_out + st_off + k * kD + 32 * p;
+          float *dst = state_out + st_off + row * kD + c0v;
 #pragma unroll
           for (int i = 0; i < 32; i += 4)
             *reinterpret_cast<float4 *>(dst + i) = make_float4(y[i], y[i + 1], y[i + 2], y[i + 3]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) y[i] *= gn_next;
+          sm100::tmem_st32(tmem + lane_off + TM_D4 + c0v, y);
         }
       }
+      if (QK == kQdqFp8Tile && (tid & 127) == 0) sm->hs[wg] = mh == 0.0f ? 0.0f : sr_tile.s;
     }
     sm100::fence_proxy_async();
     sm100::tc_fence_before();
     __syncthreads();
-    if (sm->abort) break;
+    if (tid == 0) sm->exact = QK == kQdqFp8Tile ? 1 : 0;
+    __syncthreads();
   }
 
   // An aborted CTA lets its outstanding TMA loads land (again bounded)
   // before its shared memory is released.
   if (tid == 0 && sm->abort) {
-    if (qk_pending) (void)sm100::mbar_wait(&sm->bar_qk, (uint32_t)(qk_pending - 1), kWaitNs);
-    if (v_pending) (void)sm100::mbar_wait(&sm->bar_v, (uint32_t)(v_pending - 1), kWaitNs);
+    for (int b = 0; b < 2; ++b)
+      if (sm->qk_pend[b])
+        (void)sm100::mbar_wait(&sm->bar_qk[b], (uint32_t)(sm->qk_pend[b] - 1), kWaitNs);
+    if (sm->v_pend) (void)sm100::mbar_wait(&sm->bar_v, (uint32_t)(sm->v_pend - 1), kWaitNs);
   }
   __syncthreads();
   if (warp == 0) {

