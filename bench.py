@@ -70,22 +70,24 @@ def recorded_traffic(kernel: str):
 
 
 # ------------------------------------------------------------ workload math
-def prefill_bytes(B, T, H, dk, dv, in_bytes, state_in: bool, per_key: bool) -> int:
-    """Algorithmic HBM bytes of one prefill call: q, k, v read, o written
-    (in dtype), g and beta read (fp32), state written (and read if given)."""
-    tok = B * T * H
+def prefill_bytes(tokens, n_states, H, dk, dv, in_bytes, state_in: bool, per_key: bool) -> int:
+    """Algorithmic HBM bytes of one prefill call: q, k, v read and o written
+    (in dtype), g and beta read (fp32), the states written (and read when an
+    initial state is given)."""
+    tok = tokens * H
     b = tok * (2 * dk + dv) * in_bytes + tok * dv * in_bytes
     b += tok * 4 * (dk if per_key else 1) + tok * 4
-    b += B * H * dk * dv * 4 * (2 if state_in else 1)
+    b += n_states * H * dk * dv * 4 * (2 if state_in else 1)
     return b
 
 
-def prefill_flops(B, T, H, dk, dv, C=64) -> int:
-    """Dense algorithmic flops of the chunked WY form per call: per chunk
+def prefill_flops(tokens, H, dk, dv, C=64) -> int:
+    """Dense algorithmic flops of the chunked WY form: per chunk of C tokens
     K K^T, Q K^T and W = T (bK): 3 * 2*C*C*d_k; U = T (bV) and Aqk Vn:
-    2 * 2*C*C*d_v; W H0, Q H0 and K^T Vn: 3 * 2*C*d_k*d_v."""
+    2 * 2*C*C*d_v; W H0, Q H0 and K^T Vn: 3 * 2*C*d_k*d_v; counted per
+    head-token (180,224 flop at d = 128)."""
     per_chunk = 3 * 2 * C * C * dk + 2 * 2 * C * C * dv + 3 * 2 * C * dk * dv
-    return B * H * (T // C) * per_chunk + (B * H * (T % C) * per_chunk) // C
+    return tokens * H * per_chunk // C
 
 
 def decode_bytes_per_update(dk, dv, in_bytes, per_key: bool) -> int:
@@ -225,6 +227,73 @@ def cpu_baseline_decode(case, inp, state) -> dict:
             "seconds": round(dt, 3)}
 
 
+def measure_prefill(args, dist, dev, stream, sampler, peaks, case, steps, warmup,
+                    traffic_key=None, keep=False):
+    """Time `steps` gdn_prefill calls of `case` (inputs resident in HBM).
+    Returns the result dict (and the device buffers when `keep`)."""
+    import torch
+
+    import gdn_synth as gs
+    import state_quantized_recurrence_b200 as sqr
+
+    inp = gs.generate(case)
+    d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    o = torch.empty(d["v"].shape, dtype=d["q"].dtype, device=dev)
+    st = torch.empty((case.n_seq, case.H, case.d_k, case.d_v), dtype=torch.float32, device=dev)
+
+    def step():
+        sqr.gdn_prefill_into(d["q"], d["k"], d["v"], d["g"], d["beta"], d["state_in"],
+                             d["cu_seqlens"], o, st, qdq=case.qdq)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    sqr.check_last_error(where=f"{case.name} warm-up")
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    t_wall0 = time.time()
+    ev0.record(stream)
+    for _ in range(steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    t_wall1 = time.time()
+    dist.barrier()
+    ms = ev0.elapsed_time(ev1) / steps
+    ms_max = dist.max(ms)
+    tokens = int(sum(inp["lengths"]))
+    in_bytes = 2 if case.dtype == "bf16" else 4
+    nbytes = prefill_bytes(tokens, case.n_seq, case.H, case.d_k, case.d_v, in_bytes,
+                           inp["state_in"] is not None, case.gate == "per_key")
+    flops = prefill_flops(tokens, case.H, case.d_k, case.d_v)
+    gbs = nbytes / (ms / 1e3) / 1e9
+    tfs = flops / (ms / 1e3) / 1e12
+    tc = case.dtype == "bf16" and case.gate == "scalar" and case.d_k == 128 and case.d_v == 128
+    res = {
+        "workload": f"{case.name}: n_seq={case.n_seq} H={case.H} tokens={tokens} d={case.d_k}, "
+                    f"{case.dtype}, {case.gate} gate, {case.qdq}, "
+                    f"{'random' if inp['state_in'] is not None else 'zero'} initial state",
+        "value": round(dist.world * tokens / (ms_max / 1e3), 1), "unit": "tokens/s",
+        "ms_per_step": round(ms_max, 5), "steps": steps,
+        "kernel": "tc::prefill_tc_kernel (tcgen05)" if tc else "simt::prefill_simt_kernel (FFMA)",
+        "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
+                     "traffic": (None if (args.small or traffic_key is None)
+                                 else recorded_traffic(traffic_key)),
+                     "bytes_per_launch": nbytes, "peak_source": peaks["source"],
+                     "tensor": {"achieved": round(tfs, 2), "peak": peaks["bf16_tflops"],
+                                "unit": "TFLOP/s", "frac": round(tfs / peaks["bf16_tflops"], 4),
+                                "flops_per_launch": flops}},
+        "clocks": sampler.summary(t_wall0, t_wall1),
+    }
+    if keep:
+        return res, (inp, d, o, st, step, tokens, nbytes)
+    del d, o, st
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_ours(args, dist: Dist) -> dict:
     import torch
 
@@ -249,49 +318,14 @@ def run_ours(args, dist: Dist) -> dict:
     case = gs.CONFIGS["gdn_prefill"]
     if args.small:  # same CTA count (B*H = 64), 8 chunks: for profiler captures
         case = gs.small_case("gdn_prefill", T=512)
-    inp = gs.generate(case)
-    d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
-    o = torch.empty(d["v"].shape, dtype=d["q"].dtype, device=dev)
-    st = torch.empty((case.n_seq, case.H, case.d_k, case.d_v), dtype=torch.float32, device=dev)
-
-    def step():
-        sqr.gdn_prefill_into(d["q"], d["k"], d["v"], d["g"], d["beta"], None, None, o, st,
-                             qdq=case.qdq)
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize(dev)
-    sqr.check_last_error(where="prefill warm-up")
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    dist.barrier()
-    torch.cuda.synchronize(dev)
-    t_wall0 = time.time()
-    ev0.record(stream)
-    for _ in range(args.steps):
-        step()
-    ev1.record(stream)
-    torch.cuda.synchronize(dev)
-    t_wall1 = time.time()
-    dist.barrier()
-    ms = ev0.elapsed_time(ev1) / args.steps
-    ms_max = dist.max(ms)
-    clocks = sampler.summary(t_wall0, t_wall1)
-
+    head, (inp, d, o, st, step, tokens, nbytes) = measure_prefill(
+        args, dist, dev, stream, sampler, peaks, case, args.steps, args.warmup,
+        traffic_key="prefill_tc", keep=True)
+    ms_max = head["ms_per_step"]
+    value = head["value"]
+    clocks = head["clocks"]
+    roofline = dict(head["roofline"], kernel="prefill (one launch per step)")
     B, T, H, dk, dv = case.n_seq, case.T, case.H, case.d_k, case.d_v
-    tokens = B * T
-    value = dist.world * tokens / (ms_max / 1e3)
-    nbytes = prefill_bytes(B, T, H, dk, dv, 2, False, case.gate == "per_key")
-    flops = prefill_flops(B, T, H, dk, dv)
-    gbs = nbytes / (ms / 1e3) / 1e9
-    tfs = flops / (ms / 1e3) / 1e12
-    roofline = {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
-                "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
-                "traffic": None if args.small else recorded_traffic("prefill_tc"),
-                "kernel": "prefill (one launch per step)", "bytes_per_launch": nbytes,
-                "peak_source": peaks["source"],
-                "tensor": {"achieved": round(tfs, 2), "peak": peaks["bf16_tflops"],
-                           "unit": "TFLOP/s", "frac": round(tfs / peaks["bf16_tflops"], 4),
-                           "flops_per_launch": flops}}
 
     # e2e through the C ABI from pinned host buffers (copies inside the timed region)
     e2e = None
@@ -308,6 +342,14 @@ def run_ours(args, dist: Dist) -> dict:
     if not args.no_decode:
         dec = run_decode(args, dist, dev, stream, sampler, peaks)
 
+    # ---------------- the other prefill workloads (KDA, packed varlen) ----------------
+    others = {}
+    if not args.only and not args.small and not args.no_others:
+        for name in ("kda_prefill", "varlen"):
+            c = gs.small_case(name, decode_steps=0)
+            others[name] = measure_prefill(args, dist, dev, stream, sampler, peaks, c,
+                                           max(3, min(args.steps, 10)), args.warmup)
+
     sampler.stop()
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": dist.world,
@@ -320,7 +362,7 @@ def run_ours(args, dist: Dist) -> dict:
                    "l2": f"inputs {nbytes / 1e6:.0f} MB > 126 MB L2, no flush",
                    "parallelism": f"dp{dist.world} (independent sequences per rank)"},
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps,
-        "clocks": clocks, "decode": dec, "impl": "ours",
+        "clocks": clocks, "decode": dec, "prefill_other": others or None, "impl": "ours",
     }
     dist.close()
     return res
@@ -482,6 +524,8 @@ def main():
     ap.add_argument("--only", choices=["prefill", "decode"], default=None,
                     help="measure one kernel only (profiler captures)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-others", action="store_true",
+                    help="skip the KDA and packed-varlen prefill measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--small", action="store_true", help="small case (profiling captures)")
     args = ap.parse_args()

@@ -645,7 +645,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     sm100::tc_fence_before();
     __syncthreads();
     if (sm->abort) break;
-    if (tid == 0 && !last) issue_v(tb + kC, it + 1);
+    // the next chunk's V goes to the staging slot epilogue 2 just read (issued
+    // by a warp that has no MMA to issue next)
+    if (tid == 224 && !last) issue_v(tb + kC, it + 1);
 
     // ---- MMA 3: Vn^T = R^T T^T (hi*hi + hi*lo + lo*hi), R^T from TMEM ----
     if (warp == 0) {
