@@ -41,11 +41,12 @@
 // stops, lets its in-flight TMA loads land, releases its TMEM and returns.
 #pragma once
 
-#include "gdn_common.cuh"
-#include "gdn_sm100.cuh"
+#include "gdn_tc_util.cuh"
 
 namespace gdn {
 namespace tc {
+
+using namespace tcu;
 
 constexpr int kThreads = 256;
 constexpr int kC = 64;      // chunk length
@@ -78,13 +79,6 @@ constexpr uint32_t TM_D5 = 384;   // (Aqk Vn)^T, after MMA 3  128 x 64 fp32
 constexpr uint32_t TM_VN = 448;   // Vn^T hi as A operand     128 x 64 fp16
 constexpr uint32_t TM_COLS = 512;
 
-// 16-byte aligned so that both buffers of Small::gt allow float4 loads.
-struct __align__(16) Gates {
-  float G[64], beta[64], gam[64], dec[64], ep[64], em[64];
-  float gn_exp;  // exp(G_{n-1}): decay of the chunk-start state over the chunk
-  int direct;    // 1: per-element exp of gate differences (wide gate span)
-};
-
 struct Small {
   Gates gt[2];      // gates of the current and the next chunk
   float red[2][4];  // FP8 tile amax partials per warpgroup
@@ -99,80 +93,6 @@ static_assert(sizeof(Small) <= 4096, "small-state block overflows its slot");
 static_assert(sizeof(Gates) % 16 == 0 && OFF_SMALL % 16 == 0, "gate arrays must stay 16-byte aligned");
 static_assert(OFF_P % 16 == 0 && OFF_T % 16 == 0 && (LDT * 4) % 16 == 0, "float4 rows");
 
-// Byte address of 16-byte chunk `ch` of row `r` in a 128B-swizzled tile.
-__device__ __forceinline__ uint32_t sw128(uint32_t tile, int r, int ch) {
-  return tile + (uint32_t)r * 128u + ((uint32_t)(ch ^ (r & 7)) << 4);
-}
-
-__device__ __forceinline__ uint32_t pack_h2(float a, float b) {
-  __half2 h = __floats2half2_rn(a, b);
-  return *reinterpret_cast<uint32_t *>(&h);
-}
-
-// hi = fp16(x), lo = fp16(x - hi), packed in pairs.
-__device__ __forceinline__ void split_h2(float a, float b, uint32_t &hi, uint32_t &lo) {
-  __half2 h = __floats2half2_rn(a, b);
-  float2 hf = __half22float2(h);
-  hi = *reinterpret_cast<uint32_t *>(&h);
-  lo = pack_h2(a - hf.x, b - hf.y);
-}
-
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
-                                             uint32_t d) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
-               "r"(d)
-               : "memory");
-}
-__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "r"(addr));
-  return v;
-}
-
-// 32 fp32 values -> chunks ch0 .. ch0+3 of row r of a hi and a lo tile.
-__device__ __forceinline__ void store32_hl(uint32_t thi, uint32_t tlo, int r, int ch0,
-                                           const float *x) {
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    uint32_t h0, h1, h2, h3, l0, l1, l2, l3;
-    split_h2(x[8 * c], x[8 * c + 1], h0, l0);
-    split_h2(x[8 * c + 2], x[8 * c + 3], h1, l1);
-    split_h2(x[8 * c + 4], x[8 * c + 5], h2, l2);
-    split_h2(x[8 * c + 6], x[8 * c + 7], h3, l3);
-    st_shared_v4(sw128(thi, r, ch0 + c), h0, h1, h2, h3);
-    st_shared_v4(sw128(tlo, r, ch0 + c), l0, l1, l2, l3);
-  }
-}
-
-// E4M3 codes of x0/s2 and x1/s2 (correctly rounded quotients from r = RN(1/s2),
-// Markstein's correction), returned as an fp16 pair (exact); y0, y1 receive
-// the dequantized values code * s (s = s2 unless the operands were
-// pre-scaled by a power of two).
-__device__ __forceinline__ uint32_t fp8_code_pair(float x0, float x1, float s2, float r, float &y0,
-                                                  float &y1, float s = 0.0f) {
-  const float q0 = __fmul_rn(x0, r), q1 = __fmul_rn(x1, r);
-  const float t0 = __fmaf_rn(__fmaf_rn(-q0, s2, x0), r, q0);
-  const float t1 = __fmaf_rn(__fmaf_rn(-q1, s2, x1), r, q1);
-  const __nv_fp8x2_storage_t f8 =
-      __nv_cvt_float2_to_fp8x2(make_float2(t0, t1), __NV_SATFINITE, __NV_E4M3);
-  const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(f8, __NV_E4M3);
-  const __half2 hh = *reinterpret_cast<const __half2 *>(&hr);
-  const float2 cf = __half22float2(hh);
-  const float sd = s == 0.0f ? s2 : s;
-  y0 = __fmul_rn(cf.x, sd);
-  y1 = __fmul_rn(cf.y, sd);
-  return *reinterpret_cast<const uint32_t *>(&hh);
-}
-
-__device__ __forceinline__ uint64_t kdesc(uint32_t addr) {
-  return sm100::smem_desc_sw128(addr, 16, 1024);
-}
-__device__ __forceinline__ uint64_t mndesc(uint32_t addr, uint32_t lbo) {
-  return sm100::smem_desc_sw128(addr, lbo, 1024);
-}
-
 // Bounded wait by every calling thread; a timeout marks the CTA aborted.
 __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, Small *sm,
                                               unsigned *err) {
@@ -182,43 +102,6 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, Sm
     return false;
   }
   return true;
-}
-
-// Gates of one chunk (one warp): G = inclusive cumsum of the log gates,
-// gamma = exp(G), dec = exp(G_{n-1} - G), the factors exp(+-(G - G_ref))
-// around the middle token, and beta; rows past n are zero-gated.
-__device__ __forceinline__ void load_gates(Gates *gt, const float *__restrict__ g,
-                                           const float *__restrict__ beta, long long tb, int n,
-                                           int H, int h, int lane) {
-  float x0 = lane < n ? __ldg(g + (tb + lane) * H + h) : 0.0f;
-  float x1 = lane + 32 < n ? __ldg(g + (tb + lane + 32) * H + h) : 0.0f;
-  gt->beta[lane] = lane < n ? __ldg(beta + (tb + lane) * H + h) : 0.0f;
-  gt->beta[lane + 32] = lane + 32 < n ? __ldg(beta + (tb + lane + 32) * H + h) : 0.0f;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const float y0 = __shfl_up_sync(0xffffffffu, x0, off);
-    const float y1 = __shfl_up_sync(0xffffffffu, x1, off);
-    if (lane >= off) { x0 += y0; x1 += y1; }
-  }
-  x1 += __shfl_sync(0xffffffffu, x0, 31);
-  const int rref = (n - 1) >> 1;
-  const float gref = __shfl_sync(0xffffffffu, rref < 32 ? x0 : x1, rref & 31);
-  const float gn = __shfl_sync(0xffffffffu, (n - 1) < 32 ? x0 : x1, (n - 1) & 31);
-  const float g0 = __shfl_sync(0xffffffffu, x0, 0);
-  gt->G[lane] = x0;
-  gt->G[lane + 32] = x1;
-  gt->gam[lane] = expf(x0);
-  gt->gam[lane + 32] = expf(x1);
-  gt->dec[lane] = expf(gn - x0);
-  gt->dec[lane + 32] = expf(gn - x1);
-  gt->ep[lane] = expf(x0 - gref);
-  gt->ep[lane + 32] = expf(x1 - gref);
-  gt->em[lane] = expf(gref - x0);
-  gt->em[lane + 32] = expf(gref - x1);
-  if (lane == 0) {
-    gt->gn_exp = expf(gn);
-    gt->direct = (g0 - gref > 80.0f || gref - gn > 80.0f) ? 1 : 0;
-  }
 }
 
 // In-place bf16 -> fp16 conversion of one [K;Q] buffer (16-byte chunks in
