@@ -126,4 +126,31 @@ __device__ __forceinline__ float warp_sum(float x) {
   return x;
 }
 
+
+// ------------------------------------------------------------ scheduling ----
+// Longest-first order for packed batches: the CTAs of a grid are dispatched
+// roughly in index order, so CTA group b takes the sequence whose length
+// ranks b (descending; ties by index), which lets the long sequences start
+// first and the short ones fill the tail.  Ranks are a permutation of
+// 0 .. n_seq-1 for any lengths, so exactly one sequence matches.  Called by
+// every thread of the block; needs n_seq <= blockDim.x (each of the first
+// n_seq threads ranks one candidate).
+__device__ __forceinline__ int seq_of_rank(const int *__restrict__ cu, int n_seq, int rank) {
+  __shared__ int s_pick;
+  const int t = threadIdx.x;
+  if (t == 0) s_pick = rank;
+  __syncthreads();
+  if (t < n_seq) {
+    const long long lt = (long long)cu[t + 1] - cu[t];
+    int r = 0;
+    for (int v = 0; v < n_seq; ++v) {
+      const long long lv = (long long)cu[v + 1] - cu[v];
+      r += (lv > lt) || (lv == lt && v < t);
+    }
+    if (r == rank) s_pick = t;
+  }
+  __syncthreads();
+  return s_pick;
+}
+
 }  // namespace gdn

@@ -78,8 +78,11 @@ prefill_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
 
   const int nvt = DV >> 6;
   const int vt = blockIdx.x % nvt;
-  const int unit = blockIdx.x / nvt;  // seq * H + head
-  const int h = unit % H, s = unit / H;
+  const int h = (blockIdx.x / nvt) % H;
+  int s = (blockIdx.x / nvt) / H;
+  if (cu_seqlens && (int)gridDim.x / (H * nvt) <= kThreads)  // packed: longest sequences first
+    s = seq_of_rank(cu_seqlens, (int)gridDim.x / (H * nvt), s);
+  const int unit = s * H + h;  // (sequence, head)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int rb = tid >> 4, cb = tid & 15;
 

@@ -106,22 +106,33 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, Sm
 
 // In-place bf16 -> fp16 conversion of one [K;Q] buffer (16-byte chunks in
 // their swizzled positions); rows of tokens past n are zeroed.  `nthr`
-// threads, this one being `t`.
-__device__ __forceinline__ void convert_kq(uint32_t buf, int n, int t, int nthr) {
-  for (int e = t; e < 2048; e += nthr) {
-    const int blk = e >> 10, rw = (e >> 3) & 127, ch = e & 7;
-    const uint32_t addr = buf + (uint32_t)blk * 16384u + (uint32_t)rw * 128u + (uint32_t)ch * 16u;
-    uint4 w = make_uint4(0u, 0u, 0u, 0u);
-    if ((rw & 63) < n) {
-      const uint4 src = ld_shared_v4(addr);
-      const uint32_t in[4] = {src.x, src.y, src.z, src.w};
-      uint32_t outw[4];
+// threads (a multiple of 128), this one being `t`.  Plain shared-memory
+// accesses in batches of four independent chunks, so the loads of a batch
+// are in flight together.
+__device__ __forceinline__ void convert_kq(uint8_t *buf, int n, int t, int nthr) {
+  for (int e0 = t; e0 < 2048; e0 += 4 * nthr) {
+    uint4 x[4];
+    uint8_t *ad[4];
+    bool live[4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
-        outw[j] = pack_h2(__uint_as_float(in[j] << 16), __uint_as_float(in[j] & 0xffff0000u));
-      w = make_uint4(outw[0], outw[1], outw[2], outw[3]);
+    for (int u = 0; u < 4; ++u) {
+      const int e = e0 + u * nthr;  // < 2048: 2048 is a multiple of 4 * nthr
+      const int blk = e >> 10, rw = (e >> 3) & 127, ch = e & 7;
+      ad[u] = buf + blk * 16384 + rw * 128 + ch * 16;
+      live[u] = (rw & 63) < n;
+      x[u] = *reinterpret_cast<const uint4 *>(ad[u]);
     }
-    st_shared_v4(addr, w.x, w.y, w.z, w.w);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const uint32_t in[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
+      uint32_t w[4] = {0u, 0u, 0u, 0u};
+      if (live[u]) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          w[j] = pack_h2(__uint_as_float(in[j] << 16), __uint_as_float(in[j] & 0xffff0000u));
+      }
+      *reinterpret_cast<uint4 *>(ad[u]) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
   }
 }
 
@@ -145,8 +156,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int wg = warp >> 2;                // warpgroup
   const int row = 32 * (warp & 3) + lane;  // TMEM lane = accumulator row
-  const int unit = blockIdx.x;             // seq * H + head
-  const int h = unit % H, s = unit / H;
+  const int h = blockIdx.x % H;
+  int s = blockIdx.x / H;
+  if (cu_seqlens && (int)gridDim.x / H <= kThreads)  // packed: longest sequences first
+    s = seq_of_rank(cu_seqlens, (int)gridDim.x / H, s);
+  const int unit = s * H + h;  // (sequence, head)
 
   long long t0, t1;
   if (cu_seqlens) {
@@ -269,7 +283,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   // ---- chunk 0's [K;Q]: wait, convert, MMA1 (later chunks' are prepared
   //      during the previous chunk) ----
   if (wait_or_abort(&sm->bar_qk[0], 0, sm, err) && tid == 0) sm->qk_pend[0] = 0;
-  convert_kq(base + OFF_KQ, (int)min((long long)kC, L), tid, kThreads);
+  convert_kq(gbase + OFF_KQ, (int)min((long long)kC, L), tid, kThreads);
   sm100::fence_proxy_async();
   sm100::tc_fence_before();
   __syncthreads();
@@ -292,6 +306,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     // H0's FP8 tile scale for this thread's value row (read before epilogue 4
     // overwrites it with the next chunk's scales)
     const float hsv = exact ? sm->hs[row >> 6] : 1.0f;
+    // the next chunk's raw gates, loaded now so that their latency is hidden
+    // behind this chunk's first phases (finished by warp 7 in epilogue 2)
+    GateRaw graw{};
+    if (warp == 7 && !last)
+      graw = load_gates_raw(g, beta, tb + kC, (int)min((long long)kC, L - c0 - kC), H, h, lane);
 
     // ---- MMA 2: D2 = H0^T [K;Q]^T (hi, or exact codes), + H0lo^T K^T ----
     if (warp == 0) {
@@ -505,8 +524,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         sm100::tmem_st16(tmem + lane_off + TM_RHI + 16 * half, whi);
         sm100::tmem_st16(tmem + lane_off + TM_RLO + 16 * half, wlo);
       }
-      if (warp == 7 && !last)
-        load_gates(gt_next, g, beta, tb + kC, (int)min((long long)kC, L - c0 - kC), H, h, lane);
+      if (warp == 7 && !last) finish_gates(gt_next, graw, (int)min((long long)kC, L - c0 - kC), lane);
       if (!last) {
         // Still inside WG0's solve: prepare the next chunk - convert its
         // [K;Q] (landed by TMA a chunk ago) and issue its MMA 1 (D1 was read
@@ -514,7 +532,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const int nb = kb ^ 1;
         if (wait_or_abort(&sm->bar_qk[nb], (uint32_t)(((it + 1) >> 1) & 1), sm, err) && tid == 128)
           sm->qk_pend[nb] = 0;
-        convert_kq(base + OFF_KQ + (uint32_t)nb * 32768u, (int)min((long long)kC, L - c0 - kC),
+        convert_kq(gbase + OFF_KQ + nb * 32768, (int)min((long long)kC, L - c0 - kC),
                    tid - 128, 128);
         sm100::fence_proxy_async();
         asm volatile("bar.sync 4, 128;" ::: "memory");
