@@ -292,6 +292,25 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     issue_mma1(0);
   }
 
+  // Outputs of a chunk are computed in its last epilogue but stored at the
+  // start of the next chunk (or after the loop), off the state path: 32
+  // tokens x this thread's value row, packed as bf16 pairs.
+  uint32_t opk[16];
+  __nv_bfloat16 *op_dst = nullptr;  // token 0 of the pending block, or null
+  int op_cnt = 0;                   // valid tokens in it
+  const long long op_ts = (long long)H * kD;
+  auto flush_outputs = [&]() {
+    if (op_dst) {
+#pragma unroll
+      for (int t = 0; t < 32; t += 2) {
+        const uint32_t w = opk[t >> 1];
+        if (t < op_cnt) op_dst[t * op_ts] = __ushort_as_bfloat16((unsigned short)(w & 0xffffu));
+        if (t + 1 < op_cnt) op_dst[(t + 1) * op_ts] = __ushort_as_bfloat16((unsigned short)(w >> 16));
+      }
+      op_dst = nullptr;
+    }
+  };
+
   int it = 0;
   for (long long c0 = 0; c0 < L && !sm->abort; c0 += kC, ++it) {
     const int n = (int)min((long long)kC, L - c0);
@@ -335,6 +354,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       }
       __syncwarp();
     }
+
+    flush_outputs();  // the previous chunk's outputs, while MMA 2 runs
 
     // ---- epilogue 1 (all warps; warps w and w + 4 split D1's 64 columns):
     //      rows 0-63 -> A (fp32, for the solve), rows 64-127 -> Aqk (fp16) ----
@@ -617,8 +638,6 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         float qh[32], av[32];
         sm100::tmem_ld32(tmem + lane_off + TM_D2 + 64 + 32 * wg, qh);
         sm100::tmem_ld32(tmem + lane_off + TM_D5 + 32 * wg, av);
-        __nv_bfloat16 *op = o + ((tb + 32 * wg) * H + h) * kD + row;
-        const long long ts = (long long)H * kD;
         const float sh = scale * hsv;
 #pragma unroll
         for (int t = 0; t < 32; t += 4) {
@@ -628,14 +647,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           qh[t + 2] = fmaf(sh * g4.z, qh[t + 2], scale * av[t + 2]);
           qh[t + 3] = fmaf(sh * g4.w, qh[t + 3], scale * av[t + 3]);
         }
-        if (n == kC) {
 #pragma unroll
-          for (int t = 0; t < 32; ++t) op[t * ts] = __float2bfloat16_rn(qh[t]);
-        } else {
-#pragma unroll
-          for (int t = 0; t < 32; ++t)
-            if (32 * wg + t < n) op[t * ts] = __float2bfloat16_rn(qh[t]);
+        for (int t = 0; t < 32; t += 2) {
+          __nv_bfloat162 p2 = __floats2bfloat162_rn(qh[t], qh[t + 1]);
+          opk[t >> 1] = *reinterpret_cast<uint32_t *>(&p2);
         }
+        op_cnt = n - 32 * wg;
+        op_dst = op_cnt > 0 ? o + ((tb + 32 * wg) * H + h) * kD + row : nullptr;
       }
       // H: key row `row`, value columns 64 wg .. + 63 (one FP8 tile per
       // warpgroup).  Pass 1 (FP8 tiles, INT8 groups of 64): amax of the 64
@@ -731,6 +749,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if (tid == 0) sm->exact = QK == kQdqFp8Tile ? 1 : 0;
     __syncthreads();
   }
+
+  flush_outputs();  // the last chunk's outputs
 
   // An aborted CTA lets its outstanding TMA loads land (again bounded)
   // before its shared memory is released.
