@@ -194,20 +194,25 @@ def cpu_baseline_prefill(case, inp, max_seconds: float = 12.0) -> dict:
     heads), on this host's cores; tokens/s scaled from the sample."""
     import oracle
     threads = len(os.sched_getaffinity(0))
-    T = case.T
-    done, t_total = 0, 0.0
-    for s in range(case.n_seq):
-        sl = slice(s, s + 1)
+    lengths = [int(x) for x in inp["lengths"]]
+    packed = inp["cu_seqlens"] is not None
+    done, tokens, t_total, start = 0, 0, 0.0, 0
+    for s, n in enumerate(lengths):
+        # one whole sequence (all heads): a batch row, or its packed token range
+        sl = (slice(0, 1), slice(start, start + n)) if packed else (slice(s, s + 1),)
+        st_in = inp["state_in"][s:s + 1] if inp["state_in"] is not None else None
         t0 = time.perf_counter()
         oracle.recurrence(inp["q"][sl], inp["k"][sl], inp["v"][sl], inp["g"][sl],
-                          inp["beta"][sl], None, oracle.dense_cu_seqlens(1, T),
+                          inp["beta"][sl], st_in, oracle.dense_cu_seqlens(1, n),
                           per_key_gate=case.gate == "per_key", qdq=case.qdq, n_threads=threads)
         t_total += time.perf_counter() - t0
+        start += n
         done += 1
+        tokens += n
         if t_total * (done + 1) / done > max_seconds:
             break
-    return {"value": done * T / t_total, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-            "sample": f"{done} of {case.n_seq} sequences ({T} tokens x {case.H} heads each), "
+    return {"value": tokens / t_total, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{done} of {len(lengths)} sequences ({tokens} tokens x {case.H} heads), "
                       f"fp64 token recurrence + fp32 {case.qdq} codec, OpenMP over heads",
             "seconds": round(t_total, 3)}
 
@@ -228,7 +233,7 @@ def cpu_baseline_decode(case, inp, state) -> dict:
 
 
 def measure_prefill(args, dist, dev, stream, sampler, peaks, case, steps, warmup,
-                    traffic_key=None, keep=False):
+                    traffic_key=None, keep=False, cpu=False):
     """Time `steps` gdn_prefill calls of `case` (inputs resident in HBM).
     Returns the result dict (and the device buffers when `keep`)."""
     import torch
@@ -287,6 +292,8 @@ def measure_prefill(args, dist, dev, stream, sampler, peaks, case, steps, warmup
                                 "flops_per_launch": flops}},
         "clocks": sampler.summary(t_wall0, t_wall1),
     }
+    if cpu and dist.rank == 0 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline_prefill(case, inp, max_seconds=8.0)
     if keep:
         return res, (inp, d, o, st, step, tokens, nbytes)
     del d, o, st
@@ -348,7 +355,7 @@ def run_ours(args, dist: Dist) -> dict:
         for name in ("kda_prefill", "varlen"):
             c = gs.small_case(name, decode_steps=0)
             others[name] = measure_prefill(args, dist, dev, stream, sampler, peaks, c,
-                                           max(3, min(args.steps, 10)), args.warmup)
+                                           max(3, min(args.steps, 10)), args.warmup, cpu=True)
 
     sampler.stop()
     res = {
