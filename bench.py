@@ -95,6 +95,14 @@ def decode_bytes_per_update(dk, dv, in_bytes, per_key: bool) -> int:
     return 2 * 4 * dk * dv + (2 * dk + dv) * in_bytes + dv * in_bytes + 4 * (dk if per_key else 1) + 4
 
 
+def decode_bytes_per_update_packed(dk, dv, in_bytes, per_key: bool, qdq: str) -> int:
+    """As decode_bytes_per_update with the state stored packed: one byte per
+    code plus the fp32 scales (per INT8 group / FP8 tile), read and written."""
+    n_scales = dv // 64 if qdq == "fp8_tile64" else dk * (dv // int(qdq.split("_g")[1]))
+    return (2 * dk * dv + 2 * 4 * n_scales + (2 * dk + dv) * in_bytes + dv * in_bytes
+            + 4 * (dk if per_key else 1) + 4)
+
+
 # ------------------------------------------------------------ clock sampler
 class ClockSampler:
     """nvidia-smi clock / throttle-reason samples, tagged with host time."""
@@ -345,9 +353,11 @@ def run_ours(args, dist: Dist) -> dict:
     torch.cuda.empty_cache()
 
     # ---------------- decode ----------------
-    dec = None
+    dec = dec_packed = None
     if not args.no_decode:
         dec = run_decode(args, dist, dev, stream, sampler, peaks)
+        if not args.small:
+            dec_packed = run_decode(args, dist, dev, stream, sampler, peaks, packed=True)
 
     # ---------------- the other prefill workloads (KDA, packed varlen) ----------------
     others = {}
@@ -369,7 +379,8 @@ def run_ours(args, dist: Dist) -> dict:
                    "l2": f"inputs {nbytes / 1e6:.0f} MB > 126 MB L2, no flush",
                    "parallelism": f"dp{dist.world} (independent sequences per rank)"},
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps,
-        "clocks": clocks, "decode": dec, "prefill_other": others or None, "impl": "ours",
+        "clocks": clocks, "decode": dec, "decode_packed": dec_packed,
+        "prefill_other": others or None, "impl": "ours",
     }
     dist.close()
     return res
@@ -410,7 +421,9 @@ def run_e2e(args, dist, d, o, st, step, stream, tokens) -> dict:
             "ms_per_step": round(ms_e2e, 4), "steps": e2e_steps}
 
 
-def run_decode(args, dist, dev, stream, sampler, peaks) -> dict:
+def run_decode(args, dist, dev, stream, sampler, peaks, packed: bool = False) -> dict:
+    """The serving decode workload: 512 single-token calls in one CUDA graph,
+    the state in fp32 storage, or (``packed``) as codes + scales."""
     import torch
 
     import gdn_synth as gs
@@ -424,23 +437,38 @@ def run_decode(args, dist, dev, stream, sampler, peaks) -> dict:
     dq, dk_, dv_ = inp["dec_q"].to(dev), inp["dec_k"].to(dev), inp["dec_v"].to(dev)
     dg, db = inp["dec_g"].to(dev), inp["dec_beta"].to(dev)
     state0 = inp["state_in"].to(dev)
-    state = state0.clone()
     o = torch.empty((S_steps,) + tuple(dv_.shape[1:]), dtype=dq.dtype, device=dev)
+    if packed:
+        ps0 = sqr.gdn_state_pack(state0, case.qdq)
+        ps = sqr.PackedState(ps0.codes.clone(), ps0.scales.clone(), case.qdq)
 
-    def run_all():
-        for t in range(S_steps):
-            sqr.gdn_decode_into(dq[t], dk_[t], dv_[t], dg[t], db[t], state, o[t], qdq=case.qdq)
+        def reset():
+            ps.codes.copy_(ps0.codes)
+            ps.scales.copy_(ps0.scales)
+
+        def run_all():
+            for t in range(S_steps):
+                sqr.gdn_decode_packed_into(dq[t], dk_[t], dv_[t], dg[t], db[t], ps, o[t])
+    else:
+        state = state0.clone()
+
+        def reset():
+            state.copy_(state0)
+
+        def run_all():
+            for t in range(S_steps):
+                sqr.gdn_decode_into(dq[t], dk_[t], dv_[t], dg[t], db[t], state, o[t], qdq=case.qdq)
 
     # warm-up, then capture the whole token loop in one CUDA graph
     for _ in range(max(1, args.warmup)):
-        state.copy_(state0)
+        reset()
         run_all()
     torch.cuda.synchronize(dev)
     sqr.check_last_error(where="decode warm-up")
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
         run_all()
-    state.copy_(state0)
+    reset()
     graph.replay()
     torch.cuda.synchronize(dev)
     reps = 3
@@ -458,21 +486,25 @@ def run_decode(args, dist, dev, stream, sampler, peaks) -> dict:
     ms_loop = dist.max(ev0.elapsed_time(ev1) / reps)
     updates = case.n_seq * case.H * S_steps
     ups = dist.world * updates / (ms_loop / 1e3)
-    bpu = decode_bytes_per_update(case.d_k, case.d_v, 2, False)
+    bpu = (decode_bytes_per_update_packed(case.d_k, case.d_v, 2, False, case.qdq) if packed
+           else decode_bytes_per_update(case.d_k, case.d_v, 2, False))
     ms_tok = ms_loop / S_steps
     gbs = case.n_seq * case.H * bpu / (ms_tok / 1e3) / 1e9
     cpu = None
-    if dist.world == 1 and not args.no_cpu_baseline:
+    if dist.world == 1 and not args.no_cpu_baseline and not packed:
         cpu = cpu_baseline_decode(case, inp, inp["state_in"])
     del graph
+    storage = ("packed state (1-byte codes + fp32 scales per group)" if packed
+               else "fp32 state")
     return {"metric": "QDQ-state decode updates/s", "value": round(ups, 1), "unit": "updates/s",
             "sequence_tokens_per_s": round(ups / case.H, 1),
             "workload": f"serving_decode {case.n_seq} seq x H={case.H}, d=128, bf16, "
-                        f"{case.qdq}, {S_steps} single-token calls in one CUDA graph",
+                        f"{case.qdq}, {S_steps} single-token calls in one CUDA graph, {storage}",
             "ms_per_token_step": round(ms_tok, 5), "reps": reps,
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
-                         "traffic": None if args.small else recorded_traffic("decode"),
+                         "traffic": None if args.small else recorded_traffic(
+                             "decode_packed" if packed else "decode"),
                          "bytes_per_update": bpu, "bytes_per_launch": case.n_seq * case.H * bpu,
                          "peak_source": peaks["source"]},
             "gpu_launches": S_steps * reps, "clocks": sampler.summary(t_wall0, t_wall1),

@@ -121,6 +121,45 @@ gdn_status gdn_decode(const void *q, const void *k, const void *v,
                       void *cuda_stream);
 
 /*
+ * Packed state storage.  The pages keep the QDQ'd state as fp32 values and
+ * say that compressed state storage is not part of their change (PR #2497
+ * What section); these three calls add it as a storage format of the same
+ * state.  A QDQ'd state is exactly code * scale, so a packed state holds:
+ *   codes   one byte per element, [n, H, d_k, d_v] (same order as the fp32
+ *           state): int8 codes in [-127, 127] for the INT8 modes, E4M3 bytes
+ *           (bias 7, no infinities) for GDN_QDQ_FP8_E4M3_TILE64;
+ *   scales  fp32: INT8 group G: [n, H, d_k, d_v / G] (one per key row and
+ *           group of G value columns); FP8 tile: [n, H, d_v / 64] (one per
+ *           d_k x 64 tile).  A zero group or tile has scale 0 and codes 0.
+ * Decoding a packed state gives bit-identical outputs and states to
+ * gdn_decode on the fp32 state it dequantizes to, while moving 1 + 4/G
+ * bytes per element (INT8) or 1 + 4/(64 d_k) (FP8) instead of 4.
+ * qdq must be an FP8 or INT8 mode (GDN_QDQ_NONE: GDN_ERR_UNSUPPORTED);
+ * codes and scales must be 4-byte aligned, the fp32 state 16-byte aligned.
+ *
+ * gdn_state_pack   - apply the state QDQ codec of `qdq` to fp32 states and
+ *                    store the codes and scales (the packed state then
+ *                    dequantizes to exactly QDQ(state)).
+ * gdn_state_unpack - dequantize: state = code * scale, element by element.
+ * gdn_decode_packed - gdn_decode with the state read and written packed, in
+ *                    place; the arguments are those of gdn_decode with
+ *                    state_inout replaced by (codes, scales).
+ * All three are asynchronous on cuda_stream; argument errors are returned
+ * before any launch.
+ */
+gdn_status gdn_state_pack(const float *state, void *codes, float *scales,
+                          int n, int H, int d_k, int d_v, gdn_qdq_mode qdq,
+                          void *cuda_stream);
+gdn_status gdn_state_unpack(const void *codes, const float *scales,
+                            float *state, int n, int H, int d_k, int d_v,
+                            gdn_qdq_mode qdq, void *cuda_stream);
+gdn_status gdn_decode_packed(const void *q, const void *k, const void *v,
+                             const float *g, const float *beta, void *codes,
+                             float *scales, int n_seq, int H, int d_k, int d_v,
+                             gdn_dtype dt, gdn_gate_kind gk, gdn_qdq_mode qdq,
+                             void *o, void *cuda_stream);
+
+/*
  * gdn_last_error - synchronize cuda_stream, then read and clear the current
  * device's error word.  Returns GDN_OK if no device-side error was recorded
  * since the last call, GDN_ERR_INVALID_ARG for a malformed cu_seqlens,

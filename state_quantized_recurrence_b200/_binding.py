@@ -35,6 +35,12 @@ def _load() -> ctypes.CDLL:
     L.gdn_prefill.restype = I
     L.gdn_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, P, P]
     L.gdn_decode.restype = I
+    L.gdn_decode_packed.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, P]
+    L.gdn_decode_packed.restype = I
+    L.gdn_state_pack.argtypes = [P, P, P, I, I, I, I, I, P]
+    L.gdn_state_pack.restype = I
+    L.gdn_state_unpack.argtypes = [P, P, P, I, I, I, I, I, P]
+    L.gdn_state_unpack.restype = I
     L.gdn_last_error.argtypes = [P]
     L.gdn_last_error.restype = I
     L.gdn_status_string.argtypes = [I]
@@ -158,4 +164,88 @@ def gdn_decode_into(q, k, v, g, beta, state, o, qdq: str = "int8_g32", stream=No
 def gdn_decode(q, k, v, g, beta, state, qdq: str = "int8_g32", stream=None):
     o = torch.empty(v.shape, dtype=q.dtype, device=q.device)
     gdn_decode_into(q, k, v, g, beta, state, o, qdq, stream)
+    return o
+
+
+# ------------------------------------------------------------ packed states
+class PackedState:
+    """A batch of QDQ states stored as codes + scales (see gdn_qdq.h):
+    ``codes`` uint8 [N, H, d_k, d_v] (int8 codes or E4M3 bytes), ``scales``
+    fp32 [N, H, d_k, d_v / G] (INT8 group G) or [N, H, d_v / 64] (FP8 tile)."""
+
+    def __init__(self, codes: torch.Tensor, scales: torch.Tensor, qdq: str):
+        self.codes, self.scales, self.qdq = codes, scales, qdq
+
+    @property
+    def shape(self):
+        return tuple(self.codes.shape)
+
+
+def _scales_shape(N, H, d_k, d_v, qdq: str):
+    _need(qdq in GDN_QDQ and qdq != "none", "packed states need an FP8 or INT8 qdq mode")
+    if qdq == "fp8_tile64":
+        return (N, H, d_v // 64)
+    return (N, H, d_k, d_v // int(qdq.split("_g")[1]))
+
+
+def packed_state_empty(N, H, d_k, d_v, qdq: str, device) -> PackedState:
+    return PackedState(torch.empty((N, H, d_k, d_v), dtype=torch.uint8, device=device),
+                       torch.empty(_scales_shape(N, H, d_k, d_v, qdq), dtype=torch.float32,
+                                   device=device), qdq)
+
+
+def gdn_state_pack(state: torch.Tensor, qdq: str, out: Optional[PackedState] = None,
+                   stream=None) -> PackedState:
+    """Codes and scales of QDQ(state) for fp32 ``state`` [N, H, d_k, d_v]."""
+    _need(state.dim() == 4 and state.dtype == torch.float32, "state must be fp32 [N, H, d_k, d_v]")
+    N, H, d_k, d_v = state.shape
+    ps = out if out is not None else packed_state_empty(N, H, d_k, d_v, qdq, state.device)
+    _check_dev(state, ps.codes, ps.scales)
+    _need(ps.shape == tuple(state.shape) and ps.qdq == qdq, "packed state shape / mode mismatch")
+    s = lib.gdn_state_pack(_ptr(state), _ptr(ps.codes), _ptr(ps.scales), N, H, d_k, d_v,
+                           GDN_QDQ[qdq], _stream(stream))
+    if s != 0:
+        raise GdnError(s, "gdn_state_pack")
+    return ps
+
+
+def gdn_state_unpack(ps: PackedState, out: Optional[torch.Tensor] = None, stream=None):
+    """fp32 [N, H, d_k, d_v] = code * scale."""
+    N, H, d_k, d_v = ps.shape
+    st = out if out is not None else torch.empty((N, H, d_k, d_v), dtype=torch.float32,
+                                                 device=ps.codes.device)
+    _check_dev(st, ps.codes, ps.scales)
+    s = lib.gdn_state_unpack(_ptr(ps.codes), _ptr(ps.scales), _ptr(st), N, H, d_k, d_v,
+                             GDN_QDQ[ps.qdq], _stream(stream))
+    if s != 0:
+        raise GdnError(s, "gdn_state_unpack")
+    return st
+
+
+def gdn_decode_packed_into(q, k, v, g, beta, ps: PackedState, o, stream=None) -> None:
+    """gdn_decode_into with the state stored packed (updated in place)."""
+    _check_dev(q, k, v, g, beta, ps.codes, ps.scales, o)
+    _need(q.dim() == 3 and k.shape == q.shape and v.dim() == 3 and o.shape == v.shape,
+          "q, k [N, H, d_k]; v, o [N, H, d_v]")
+    N, H, d_k = q.shape
+    d_v = v.shape[-1]
+    _need(q.dtype in GDN_DTYPE and k.dtype == q.dtype and v.dtype == q.dtype and o.dtype == q.dtype,
+          "q, k, v, o must share dtype bf16 or fp32")
+    _need(g.dtype == torch.float32 and beta.dtype == torch.float32 and beta.shape == (N, H),
+          "g, beta must be fp32; beta [N, H]")
+    gk = _gate_kind(g, 2)
+    _need(g.shape == ((N, H) if gk == "scalar" else (N, H, d_k)), "g must be [N,H] or [N,H,d_k]")
+    _need(ps.shape == (N, H, d_k, d_v) and ps.codes.dtype == torch.uint8 and
+          tuple(ps.scales.shape) == _scales_shape(N, H, d_k, d_v, ps.qdq),
+          "packed state does not match the call")
+    s = lib.gdn_decode_packed(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(ps.codes),
+                              _ptr(ps.scales), N, H, d_k, d_v, GDN_DTYPE[q.dtype], GDN_GATE[gk],
+                              GDN_QDQ[ps.qdq], _ptr(o), _stream(stream))
+    if s != 0:
+        raise GdnError(s, "gdn_decode_packed")
+
+
+def gdn_decode_packed(q, k, v, g, beta, ps: PackedState, stream=None):
+    o = torch.empty(v.shape, dtype=q.dtype, device=q.device)
+    gdn_decode_packed_into(q, k, v, g, beta, ps, o, stream)
     return o

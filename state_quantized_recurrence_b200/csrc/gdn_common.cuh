@@ -109,6 +109,23 @@ __device__ __forceinline__ float2 qdq_fp8_2(float x0, float x1, const ScaleRecip
   return make_float2(__fmul_rn(c.x, sr.s), __fmul_rn(c.y, sr.s));
 }
 
+// The codes themselves (for packed state storage); the dequantized values
+// of the functions above are exactly code * s.
+__device__ __forceinline__ float int8_code(float x, const ScaleRecip &sr) {
+  return fminf(fmaxf(rintf(div_by_scale(x, sr)), -127.0f), 127.0f);
+}
+// E4M3 bytes of x0 / s and x1 / s (x0 in the low byte).
+__device__ __forceinline__ unsigned short e4m3_code2(float x0, float x1, const ScaleRecip &sr) {
+  return (unsigned short)__nv_cvt_float2_to_fp8x2(make_float2(div_by_scale(x0, sr), div_by_scale(x1, sr)),
+                                                  __NV_SATFINITE, __NV_E4M3);
+}
+// Two E4M3 bytes (low byte first) -> their values, exactly.
+__device__ __forceinline__ float2 e4m3_pair_to_f2(unsigned short p) {
+  __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)p, __NV_E4M3);
+  __half2 hh = *reinterpret_cast<__half2 *>(&h);
+  return __half22float2(hh);
+}
+
 __device__ __forceinline__ float int8_scale(float amax) { return __fdiv_rn(amax, 127.0f); }
 __device__ __forceinline__ float fp8_scale(float amax) { return __fdiv_rn(amax, 448.0f); }
 

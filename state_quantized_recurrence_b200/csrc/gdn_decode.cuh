@@ -10,60 +10,166 @@
 //   H  = QDQ(H)                   (after every decode token)
 //
 // with H = S^T stored [d_k, d_v].  The path is HBM-bound: each call reads and
-// writes every state once (2 * 4 * d_k * d_v bytes per head), so the kernel
-// streams the state once with coalesced 128-bit loads and stores, keeps it in
-// registers across the two key-axis reductions, and writes it back in place.
+// writes every state once, so the kernel streams the state once with
+// coalesced loads and stores, keeps it in registers across the two key-axis
+// reductions, and writes it back in place.
+//
+// Two state storages share the kernel:
+//   fp32    the QDQ'd values, 4 bytes per element (the pages' layout);
+//   packed  the codes of the same QDQ (int8, or E4M3 bytes) plus one fp32
+//           scale per INT8 group / FP8 tile.  code * scale is exactly the
+//           fp32 value the other storage holds, so both give bit-identical
+//           results, with 1 + 4/group bytes per element moved instead of 4.
+//           (The pages keep fp32 storage and mark compressed storage as not
+//           done, PR #2497 What section; it is an added interface.)
 //
 // Work split: one 256-thread CTA per (sequence, head, 64-column value tile),
-// i.e. a d_k x 64 fp32 slab (32 KB at d_k = 128) - exactly one FP8 scale
-// tile.  Thread t owns columns 4*(t % 16) .. +3 of rows (t / 16) + 16 j, so a
-// warp reads two full 256-byte row segments per load instruction, an INT8
-// group of 32 columns lives in 8 consecutive lanes, and the key-axis
-// reductions are one xor-16 shuffle plus an 8-warp shared-memory pass.
+// i.e. a d_k x 64 slab - exactly one FP8 scale tile.  Thread t owns columns
+// 4*(t % 16) .. +3 of rows (t / 16) + 16 j, so a warp reads two full row
+// segments per load instruction, an INT8 group of 32 columns lives in 8
+// consecutive lanes, and the key-axis reductions are one xor-16 shuffle plus
+// an 8-warp shared-memory pass.
 #pragma once
 
 #include "gdn_common.cuh"
 
 namespace gdn {
 
-// QK: kQdqNone / kQdqFp8Tile / kQdqInt8; GROUP: INT8 group width (16/32/64).
-// 256 threads and <= 80 registers per thread give 3 CTAs (96 KB of state
-// loads in flight) per SM; k, q and the per-key decays sit in shared memory
-// so the 32 state values are the only large register footprint.
-template <typename Tin, int DK, int DV, bool PER_KEY, int QK, int GROUP>
-__global__ void __launch_bounds__(256, 3)
-decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
-              const Tin *__restrict__ v, const float *__restrict__ g,
-              const float *__restrict__ beta, float *__restrict__ state,
-              Tin *__restrict__ o, float scale) {
-  constexpr int RPT = DK / 16;  // state rows per thread
-  __shared__ float s_k[DK], s_q[DK], s_al[PER_KEY ? DK : 1];
-  __shared__ float4 red_a[8][16], red_b[8][16];
-  __shared__ float red_m[8];
+// Where the state of one (sequence, head) lives.
+struct StateRef {
+  float *vals;     // fp32 storage: [d_k, d_v]
+  uint8_t *codes;  // packed storage: [d_k, d_v] one byte per element
+  float *scales;   // packed storage: INT8 [d_k, d_v / GROUP], FP8 [d_v / 64]
+};
 
-  constexpr int nvt = DV / 64;
-  const long long unit = blockIdx.x / nvt;  // sequence * H + head
-  const int vt = blockIdx.x - (int)(unit * nvt);
+template <int DK, int DV, int QK, int GROUP, bool PACKED>
+struct StateIO {
+  static constexpr int RPT = DK / 16;  // state rows per thread
+
+  // Row `r`, columns col .. col+3 of the state, as fp32 values.
+  __device__ __forceinline__ static void load(const StateRef &sr, int rg, int col, float4 (&h)[RPT]) {
+    if (!PACKED) {
+#pragma unroll
+      for (int j = 0; j < RPT; ++j)
+        h[j] = __ldcs(reinterpret_cast<const float4 *>(sr.vals + (rg + 16 * j) * DV + col));
+    } else {
+      uint32_t cw[RPT];
+      float s[RPT];
+#pragma unroll
+      for (int j = 0; j < RPT; ++j)
+        cw[j] = __ldcs(reinterpret_cast<const unsigned int *>(sr.codes + (rg + 16 * j) * DV + col));
+      if (QK == kQdqInt8) {
+#pragma unroll
+        for (int j = 0; j < RPT; ++j) s[j] = __ldg(sr.scales + (rg + 16 * j) * (DV / GROUP) + col / GROUP);
+#pragma unroll
+        for (int j = 0; j < RPT; ++j) {
+          const uint32_t w = cw[j];
+          h[j] = make_float4(__fmul_rn((float)(int8_t)(w & 0xffu), s[j]),
+                             __fmul_rn((float)(int8_t)((w >> 8) & 0xffu), s[j]),
+                             __fmul_rn((float)(int8_t)((w >> 16) & 0xffu), s[j]),
+                             __fmul_rn((float)(int8_t)(w >> 24), s[j]));
+        }
+      } else {
+        const float st = __ldg(sr.scales + col / 64);
+#pragma unroll
+        for (int j = 0; j < RPT; ++j) {
+          const float2 lo = e4m3_pair_to_f2((unsigned short)(cw[j] & 0xffffu));
+          const float2 hi = e4m3_pair_to_f2((unsigned short)(cw[j] >> 16));
+          h[j] = make_float4(__fmul_rn(lo.x, st), __fmul_rn(lo.y, st), __fmul_rn(hi.x, st),
+                             __fmul_rn(hi.y, st));
+        }
+      }
+    }
+  }
+
+  // QDQ of the slab and store: fp32 values, or codes + scales.  `red` is 8
+  // floats of shared memory (FP8 tile amax); called by all 256 threads.
+  __device__ __forceinline__ static void qdq_store(const StateRef &sr, int rg, int col, int lane,
+                                                   int warp, float *red, float4 (&h)[RPT]) {
+    uint32_t cw[RPT];  // packed codes, 4 per row
+    if (QK == kQdqInt8) {
+#pragma unroll
+      for (int j = 0; j < RPT; ++j) {
+        float m = fmaxf(fmaxf(fabsf(h[j].x), fabsf(h[j].y)), fmaxf(fabsf(h[j].z), fabsf(h[j].w)));
+        m = group_max<GROUP / 4>(m);  // a group spans GROUP / 4 consecutive lanes
+        float sc = 0.0f;
+        if (m == 0.0f) {
+          h[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+          cw[j] = 0u;
+        } else {
+          const ScaleRecip s = make_scale(int8_scale(m));
+          sc = s.s;
+          if (PACKED) {
+            const float c0 = int8_code(h[j].x, s), c1 = int8_code(h[j].y, s),
+                        c2 = int8_code(h[j].z, s), c3 = int8_code(h[j].w, s);
+            cw[j] = ((uint32_t)(uint8_t)(int8_t)c0) | ((uint32_t)(uint8_t)(int8_t)c1 << 8) |
+                    ((uint32_t)(uint8_t)(int8_t)c2 << 16) | ((uint32_t)(uint8_t)(int8_t)c3 << 24);
+          } else {
+            h[j].x = qdq_int8(h[j].x, s); h[j].y = qdq_int8(h[j].y, s);
+            h[j].z = qdq_int8(h[j].z, s); h[j].w = qdq_int8(h[j].w, s);
+          }
+        }
+        if (PACKED && (col % GROUP) == 0)
+          sr.scales[(rg + 16 * j) * (DV / GROUP) + col / GROUP] = sc;
+      }
+    } else if (QK == kQdqFp8Tile) {
+      float m = 0.0f;
+#pragma unroll
+      for (int j = 0; j < RPT; ++j)
+        m = fmaxf(m, fmaxf(fmaxf(fabsf(h[j].x), fabsf(h[j].y)), fmaxf(fabsf(h[j].z), fabsf(h[j].w))));
+      m = group_max<32>(m);
+      if (lane == 0) red[warp] = m;
+      __syncthreads();
+      m = red[0];
+#pragma unroll
+      for (int w = 1; w < 8; ++w) m = fmaxf(m, red[w]);
+      if (m == 0.0f) {
+#pragma unroll
+        for (int j = 0; j < RPT; ++j) {
+          h[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+          cw[j] = 0u;
+        }
+      } else {
+        const ScaleRecip s = make_scale(fp8_scale(m));
+#pragma unroll
+        for (int j = 0; j < RPT; ++j) {
+          if (PACKED) {
+            cw[j] = (uint32_t)e4m3_code2(h[j].x, h[j].y, s) | ((uint32_t)e4m3_code2(h[j].z, h[j].w, s) << 16);
+          } else {
+            const float2 lo = qdq_fp8_2(h[j].x, h[j].y, s);
+            const float2 hi = qdq_fp8_2(h[j].z, h[j].w, s);
+            h[j] = make_float4(lo.x, lo.y, hi.x, hi.y);
+          }
+        }
+      }
+      if (PACKED && rg == 0 && (col % 64) == 0) sr.scales[col / 64] = m == 0.0f ? 0.0f : fp8_scale(m);
+    }
+    if (!PACKED) {
+#pragma unroll
+      for (int j = 0; j < RPT; ++j)
+        __stcs(reinterpret_cast<float4 *>(sr.vals + (rg + 16 * j) * DV + col), h[j]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < RPT; ++j)
+        __stcs(reinterpret_cast<unsigned int *>(sr.codes + (rg + 16 * j) * DV + col), cw[j]);
+    }
+  }
+};
+
+// The token update of one slab once its state (h), k, q, the decays and v
+// are staged: decay, the key-axis reductions, the output, the delta update,
+// the QDQ and the store.  Shared by both decode kernels, so the fp32 and the
+// packed storage run the same arithmetic.
+template <typename Tin, int DK, int DV, bool PER_KEY, int QK, int GROUP, bool PACKED>
+__device__ __forceinline__ void decode_slab(float4 (&h)[DK / 16], const float *s_k,
+                                            const float *s_q, const float *s_al, float a_scalar,
+                                            float bt, float4 v4, float4 (*red_a)[16],
+                                            float4 (*red_b)[16], float *red_m, const StateRef &sr,
+                                            Tin *__restrict__ o_row, int col, float scale) {
+  using IO = StateIO<DK, DV, QK, GROUP, PACKED>;
+  constexpr int RPT = IO::RPT;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int cq = tid & 15, rg = tid >> 4;
-  const int col = vt * 64 + cq * 4;
-
-  float *S = state + unit * (long long)(DK * DV) + (rg * DV + col);
-  // Issue the state loads first: they are the only HBM-sized traffic.
-  float4 h[RPT];
-#pragma unroll
-  for (int j = 0; j < RPT; ++j)
-    h[j] = __ldcs(reinterpret_cast<const float4 *>(S + 16 * j * DV));
-
-  if (tid < DK) {
-    s_k[tid] = to_f32(k[unit * DK + tid]);
-    s_q[tid] = to_f32(q[unit * DK + tid]);
-    if (PER_KEY) s_al[tid] = expf(__ldg(g + unit * DK + tid));
-  }
-  const float bt = __ldg(beta + unit);
-  const float a_scalar = PER_KEY ? 0.0f : expf(__ldg(g + unit));
-  const float4 v4 = load4(v + unit * DV + col);
-  __syncthreads();
 
   // k^T q, computed redundantly by every warp from shared memory.
   float kq = 0.0f;
@@ -102,7 +208,7 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
   u[0] = bt * (v4.x - a[0]); u[1] = bt * (v4.y - a[1]);
   u[2] = bt * (v4.z - a[2]); u[3] = bt * (v4.w - a[3]);
   if (rg == 0)
-    store4(o + unit * DV + col, scale * fmaf(kq, u[0], b[0]), scale * fmaf(kq, u[1], b[1]),
+    store4(o_row + col, scale * fmaf(kq, u[0], b[0]), scale * fmaf(kq, u[1], b[1]),
            scale * fmaf(kq, u[2], b[2]), scale * fmaf(kq, u[3], b[3]));
 
   // Delta update H = Ht + k u^T.
@@ -113,48 +219,91 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
     h[j].z = fmaf(kr, u[2], h[j].z); h[j].w = fmaf(kr, u[3], h[j].w);
   }
 
-  // State QDQ.
-  if (QK == kQdqInt8) {
-#pragma unroll
-    for (int j = 0; j < RPT; ++j) {
-      float m = fmaxf(fmaxf(fabsf(h[j].x), fabsf(h[j].y)), fmaxf(fabsf(h[j].z), fabsf(h[j].w)));
-      m = group_max<GROUP / 4>(m);  // a group spans GROUP / 4 consecutive lanes
-      if (m == 0.0f) {
-        h[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-      } else {
-        const ScaleRecip sr = make_scale(int8_scale(m));
-        h[j].x = qdq_int8(h[j].x, sr); h[j].y = qdq_int8(h[j].y, sr);
-        h[j].z = qdq_int8(h[j].z, sr); h[j].w = qdq_int8(h[j].w, sr);
-      }
-    }
-  } else if (QK == kQdqFp8Tile) {
-    float m = 0.0f;
-#pragma unroll
-    for (int j = 0; j < RPT; ++j)
-      m = fmaxf(m, fmaxf(fmaxf(fabsf(h[j].x), fabsf(h[j].y)), fmaxf(fabsf(h[j].z), fabsf(h[j].w))));
-    m = group_max<32>(m);
-    if (lane == 0) red_m[warp] = m;
-    __syncthreads();
-    m = red_m[0];
-#pragma unroll
-    for (int w = 1; w < 8; ++w) m = fmaxf(m, red_m[w]);
-    if (m == 0.0f) {
-#pragma unroll
-      for (int j = 0; j < RPT; ++j) h[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-    } else {
-      const ScaleRecip sr = make_scale(fp8_scale(m));
-#pragma unroll
-      for (int j = 0; j < RPT; ++j) {
-        const float2 lo = qdq_fp8_2(h[j].x, h[j].y, sr);
-        const float2 hi = qdq_fp8_2(h[j].z, h[j].w, sr);
-        h[j] = make_float4(lo.x, lo.y, hi.x, hi.y);
-      }
-    }
-  }
+  // State QDQ and store.
+  IO::qdq_store(sr, rg, col, lane, warp, red_m, h);
+}
 
+__device__ __forceinline__ StateRef state_ref(float *state, uint8_t *codes, float *scales,
+                                              long long unit, int dk_dv, int n_scales) {
+  StateRef sr;
+  sr.vals = state ? state + unit * (long long)dk_dv : nullptr;
+  sr.codes = codes ? codes + unit * (long long)dk_dv : nullptr;
+  sr.scales = scales ? scales + unit * (long long)n_scales : nullptr;
+  return sr;
+}
+
+// One 256-thread CTA per slab.  QK: kQdqNone / kQdqFp8Tile / kQdqInt8;
+// GROUP: INT8 group width (16/32/64); PACKED: the state is stored as codes +
+// scales (QK != kQdqNone).  k, q and the per-key decays sit in shared memory
+// so the state values are the only large register footprint: <= 80
+// registers give 3 CTAs per SM (96 KB of fp32 state loads in flight); the
+// packed kernel, which moves 3.5x fewer bytes per slab and is bound by its
+// arithmetic, runs 4 CTAs per SM (<= 64 registers).
+template <typename Tin, int DK, int DV, bool PER_KEY, int QK, int GROUP, bool PACKED>
+__global__ void __launch_bounds__(256, PACKED ? 4 : 3)
+decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
+              const Tin *__restrict__ v, const float *__restrict__ g,
+              const float *__restrict__ beta, float *__restrict__ state,
+              uint8_t *__restrict__ codes, float *__restrict__ scales,
+              Tin *__restrict__ o, float scale) {
+  using IO = StateIO<DK, DV, QK, GROUP, PACKED>;
+  constexpr int NSC = QK == kQdqInt8 ? DK * (DV / GROUP) : DV / 64;  // scales per state
+  __shared__ float s_k[DK], s_q[DK], s_al[PER_KEY ? DK : 1];
+  __shared__ float4 red_a[8][16], red_b[8][16];
+  __shared__ float red_m[8];
+
+  constexpr int nvt = DV / 64;
+  const long long unit = blockIdx.x / nvt;  // sequence * H + head
+  const int vt = blockIdx.x - (int)(unit * nvt);
+  const int tid = threadIdx.x;
+  const int col = vt * 64 + (tid & 15) * 4, rg = tid >> 4;
+
+  const StateRef sr = state_ref(state, codes, scales, unit, DK * DV, NSC);
+  // Issue the state loads first: they are the only HBM-sized traffic.
+  float4 h[IO::RPT];
+  IO::load(sr, rg, col, h);
+
+  if (tid < DK) {
+    s_k[tid] = to_f32(k[unit * DK + tid]);
+    s_q[tid] = to_f32(q[unit * DK + tid]);
+    if (PER_KEY) s_al[tid] = expf(__ldg(g + unit * DK + tid));
+  }
+  const float bt = __ldg(beta + unit);
+  const float a_scalar = PER_KEY ? 0.0f : expf(__ldg(g + unit));
+  const float4 v4 = load4(v + unit * DV + col);
+  __syncthreads();
+  decode_slab<Tin, DK, DV, PER_KEY, QK, GROUP, PACKED>(h, s_k, s_q, s_al, a_scalar, bt, v4, red_a,
+                                                       red_b, red_m, sr, o + unit * DV, col, scale);
+}
+
+// Conversion between the two storages of a state batch [n, d_k, d_v]: pack
+// applies the QDQ codec to fp32 states and stores codes + scales (the packed
+// state then dequantizes to exactly the QDQ'd values); unpack dequantizes.
+template <int DK, int DV, int QK, int GROUP, bool TO_PACKED>
+__global__ void __launch_bounds__(256, 3)
+state_convert_kernel(float *__restrict__ state, uint8_t *__restrict__ codes,
+                     float *__restrict__ scales) {
+  constexpr int nvt = DV / 64;
+  const long long unit = blockIdx.x / nvt;
+  const int vt = blockIdx.x - (int)(unit * nvt);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int cq = tid & 15, rg = tid >> 4;
+  const int col = vt * 64 + cq * 4;
+  __shared__ float red_m[8];
+  StateRef sr;
+  sr.vals = state + unit * (long long)(DK * DV);
+  sr.codes = codes + unit * (long long)(DK * DV);
+  sr.scales = scales + unit * (long long)(QK == kQdqInt8 ? DK * (DV / GROUP) : DV / 64);
+  float4 h[DK / 16];
+  if (TO_PACKED) {
+    StateIO<DK, DV, QK, GROUP, false>::load(sr, rg, col, h);
+    StateIO<DK, DV, QK, GROUP, true>::qdq_store(sr, rg, col, lane, warp, red_m, h);
+  } else {
+    StateIO<DK, DV, QK, GROUP, true>::load(sr, rg, col, h);
 #pragma unroll
-  for (int j = 0; j < RPT; ++j)
-    __stcs(reinterpret_cast<float4 *>(S + 16 * j * DV), h[j]);
+    for (int j = 0; j < DK / 16; ++j)
+      *reinterpret_cast<float4 *>(sr.vals + (rg + 16 * j) * DV + col) = h[j];
+  }
 }
 
 }  // namespace gdn

@@ -69,12 +69,33 @@ gdn_status check_common(const void *q, const void *k, const void *v, const float
   return GDN_OK;
 }
 
+// State storage of a decode call: fp32 values, or packed codes + scales.
+struct StateArgs {
+  float *vals;
+  uint8_t *codes;
+  float *scales;
+  bool packed;
+};
+
+template <typename Tin, int DK, int DV, bool PK, int QK, int GR>
+void decode_launch_one(dim3 grid, cudaStream_t st, const Tin *q, const Tin *k, const Tin *v,
+                       const float *g, const float *beta, const StateArgs &sa, Tin *o,
+                       float scale) {
+  if (sa.packed) {
+    if constexpr (QK != gdn::kQdqNone)
+      gdn::decode_kernel<Tin, DK, DV, PK, QK, GR, true><<<grid, 256, 0, st>>>(
+          q, k, v, g, beta, nullptr, sa.codes, sa.scales, o, scale);
+  } else {
+    gdn::decode_kernel<Tin, DK, DV, PK, QK, GR, false><<<grid, 256, 0, st>>>(
+        q, k, v, g, beta, sa.vals, nullptr, nullptr, o, scale);
+  }
+}
+
 template <typename Tin, int DK, int DV, bool PK>
 void decode_dispatch(dim3 grid, cudaStream_t st, const Tin *q, const Tin *k, const Tin *v,
-                     const float *g, const float *beta, float *state, Tin *o, float scale,
+                     const float *g, const float *beta, const StateArgs &sa, Tin *o, float scale,
                      int kind, int group) {
-#define GDN_DEC(QK, GR) \
-  gdn::decode_kernel<Tin, DK, DV, PK, QK, GR><<<grid, 256, 0, st>>>(q, k, v, g, beta, state, o, scale)
+#define GDN_DEC(QK, GR) decode_launch_one<Tin, DK, DV, PK, QK, GR>(grid, st, q, k, v, g, beta, sa, o, scale)
   if (kind == gdn::kQdqNone) GDN_DEC(gdn::kQdqNone, 32);
   else if (kind == gdn::kQdqFp8Tile) GDN_DEC(gdn::kQdqFp8Tile, 32);
   else if (group == 16) GDN_DEC(gdn::kQdqInt8, 16);
@@ -85,15 +106,15 @@ void decode_dispatch(dim3 grid, cudaStream_t st, const Tin *q, const Tin *k, con
 
 template <typename Tin, int DK, int DV>
 void decode_dispatch_gate(bool per_key, dim3 grid, cudaStream_t st, const Tin *q, const Tin *k,
-                          const Tin *v, const float *g, const float *beta, float *state, Tin *o,
-                          float scale, int kind, int group) {
-  if (per_key) decode_dispatch<Tin, DK, DV, true>(grid, st, q, k, v, g, beta, state, o, scale, kind, group);
-  else decode_dispatch<Tin, DK, DV, false>(grid, st, q, k, v, g, beta, state, o, scale, kind, group);
+                          const Tin *v, const float *g, const float *beta, const StateArgs &sa,
+                          Tin *o, float scale, int kind, int group) {
+  if (per_key) decode_dispatch<Tin, DK, DV, true>(grid, st, q, k, v, g, beta, sa, o, scale, kind, group);
+  else decode_dispatch<Tin, DK, DV, false>(grid, st, q, k, v, g, beta, sa, o, scale, kind, group);
 }
 
 template <typename Tin>
 gdn_status launch_decode(const void *q, const void *k, const void *v, const float *g,
-                         const float *beta, float *state, int n_seq, int H, int d_k,
+                         const float *beta, const StateArgs &state, int n_seq, int H, int d_k,
                          int d_v, bool per_key, int kind, int group, void *o,
                          cudaStream_t st) {
   const long long blocks = (long long)n_seq * H * (d_v / 64);
@@ -123,6 +144,31 @@ gdn_status launch_simt_one(const Tin *q, const Tin *k, const Tin *v, const float
     return GDN_ERR_CUDA;
   kern<<<blocks, gdn::simt::kThreads, L::kBytes, st>>>(q, k, v, g, beta, state_in, cu, T, H, d_v,
                                                        scale, kind, group, o, state_out, err);
+  return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+template <int DK, int DV, bool TO>
+void convert_dispatch(dim3 grid, cudaStream_t st, float *vals, uint8_t *codes, float *scales,
+                      int kind, int group) {
+#define GDN_CV(QK, GR) gdn::state_convert_kernel<DK, DV, QK, GR, TO><<<grid, 256, 0, st>>>(vals, codes, scales)
+  if (kind == gdn::kQdqFp8Tile) GDN_CV(gdn::kQdqFp8Tile, 32);
+  else if (group == 16) GDN_CV(gdn::kQdqInt8, 16);
+  else if (group == 64) GDN_CV(gdn::kQdqInt8, 64);
+  else GDN_CV(gdn::kQdqInt8, 32);
+#undef GDN_CV
+}
+
+gdn_status launch_convert(float *vals, uint8_t *codes, float *scales, int n, int H, int d_k,
+                          int d_v, int kind, int group, bool to_packed, cudaStream_t st) {
+  const long long blocks = (long long)n * H * (d_v / 64);
+  if (blocks > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+  dim3 grid((unsigned)blocks);
+#define GDN_CVD(DK, DV) \
+  (to_packed ? convert_dispatch<DK, DV, true>(grid, st, vals, codes, scales, kind, group) \
+             : convert_dispatch<DK, DV, false>(grid, st, vals, codes, scales, kind, group))
+  if (d_k == 128) { if (d_v == 128) GDN_CVD(128, 128); else GDN_CVD(128, 64); }
+  else            { if (d_v == 128) GDN_CVD(64, 128);  else GDN_CVD(64, 64); }
+#undef GDN_CVD
   return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
@@ -249,11 +295,57 @@ gdn_status gdn_decode(const void *q, const void *k, const void *v, const float *
   if (!state_inout || !aligned(state_inout, 16)) return GDN_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
   const bool pk = gk == GDN_GATE_PER_KEY;
+  const StateArgs sa{state_inout, nullptr, nullptr, false};
   if (dt == GDN_DTYPE_BF16)
-    return launch_decode<__nv_bfloat16>(q, k, v, g, beta, state_inout, n_seq, H, d_k, d_v, pk,
-                                        kind, group, o, st);
-  return launch_decode<float>(q, k, v, g, beta, state_inout, n_seq, H, d_k, d_v, pk, kind,
-                              group, o, st);
+    return launch_decode<__nv_bfloat16>(q, k, v, g, beta, sa, n_seq, H, d_k, d_v, pk, kind,
+                                        group, o, st);
+  return launch_decode<float>(q, k, v, g, beta, sa, n_seq, H, d_k, d_v, pk, kind, group, o, st);
+}
+
+gdn_status gdn_decode_packed(const void *q, const void *k, const void *v, const float *g,
+                             const float *beta, void *codes, float *scales, int n_seq, int H,
+                             int d_k, int d_v, gdn_dtype dt, gdn_gate_kind gk, gdn_qdq_mode qdq,
+                             void *o, void *cuda_stream) {
+  gdn_status s = check_common(q, k, v, g, beta, o, n_seq, H, d_k, d_v, dt, gk, qdq, n_seq);
+  if (s != GDN_OK) return s;
+  int kind = 0, group = 32;
+  if (!qdq_params(qdq, d_v, &kind, &group) || kind == gdn::kQdqNone) return GDN_ERR_UNSUPPORTED;
+  if (n_seq == 0) return GDN_OK;
+  if (!codes || !scales || !aligned(codes, 4) || !aligned(scales, 4)) return GDN_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  const bool pk = gk == GDN_GATE_PER_KEY;
+  const StateArgs sa{nullptr, static_cast<uint8_t *>(codes), scales, true};
+  if (dt == GDN_DTYPE_BF16)
+    return launch_decode<__nv_bfloat16>(q, k, v, g, beta, sa, n_seq, H, d_k, d_v, pk, kind,
+                                        group, o, st);
+  return launch_decode<float>(q, k, v, g, beta, sa, n_seq, H, d_k, d_v, pk, kind, group, o, st);
+}
+
+static gdn_status state_convert(float *state, void *codes, float *scales, int n, int H, int d_k,
+                                int d_v, gdn_qdq_mode qdq, bool to_packed, void *cuda_stream) {
+  if (n < 0 || H <= 0) return GDN_ERR_INVALID_ARG;
+  if ((d_k != 64 && d_k != 128) || (d_v != 64 && d_v != 128)) return GDN_ERR_UNSUPPORTED;
+  if ((unsigned)qdq > (unsigned)GDN_QDQ_INT8_GROUP64) return GDN_ERR_UNSUPPORTED;
+  int kind = 0, group = 32;
+  if (!qdq_params(qdq, d_v, &kind, &group) || kind == gdn::kQdqNone) return GDN_ERR_UNSUPPORTED;
+  if (n == 0) return GDN_OK;
+  if (!state || !codes || !scales || !aligned(state, 16) || !aligned(codes, 4) ||
+      !aligned(scales, 4))
+    return GDN_ERR_INVALID_ARG;
+  return launch_convert(state, static_cast<uint8_t *>(codes), scales, n, H, d_k, d_v, kind, group,
+                        to_packed, static_cast<cudaStream_t>(cuda_stream));
+}
+
+gdn_status gdn_state_pack(const float *state, void *codes, float *scales, int n, int H, int d_k,
+                          int d_v, gdn_qdq_mode qdq, void *cuda_stream) {
+  return state_convert(const_cast<float *>(state), codes, scales, n, H, d_k, d_v, qdq, true,
+                       cuda_stream);
+}
+
+gdn_status gdn_state_unpack(const void *codes, const float *scales, float *state, int n, int H,
+                            int d_k, int d_v, gdn_qdq_mode qdq, void *cuda_stream) {
+  return state_convert(state, const_cast<void *>(codes), const_cast<float *>(scales), n, H, d_k,
+                       d_v, qdq, false, cuda_stream);
 }
 
 gdn_status gdn_prefill(const void *q, const void *k, const void *v, const float *g,

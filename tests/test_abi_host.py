@@ -33,6 +33,11 @@ def lib():
     L.gdn_prefill.restype = I
     L.gdn_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, P, P]
     L.gdn_decode.restype = I
+    L.gdn_decode_packed.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, P]
+    L.gdn_decode_packed.restype = I
+    for f in (L.gdn_state_pack, L.gdn_state_unpack):
+        f.argtypes = [P, P, P, I, I, I, I, I, P]
+        f.restype = I
     L.gdn_status_string.argtypes = [I]
     L.gdn_status_string.restype = ctypes.c_char_p
     return L
@@ -86,7 +91,26 @@ def dc(lib, **kw):
                           a["stream"])
 
 
-@pytest.mark.parametrize("call", [pf, dc])
+def dp(lib, **kw):
+    a = dict(q=A, k=A, v=A, g=A, beta=A, codes=A, scales=A, n_seq=2, H=4, d_k=128, d_v=128,
+             dt=BF16, gk=0, qdq=2, o=A, stream=None)
+    a.update(kw)
+    return lib.gdn_decode_packed(a["q"], a["k"], a["v"], a["g"], a["beta"], a["codes"],
+                                 a["scales"], a["n_seq"], a["H"], a["d_k"], a["d_v"], a["dt"],
+                                 a["gk"], a["qdq"], a["o"], a["stream"])
+
+
+def cv(lib, unpack=False, **kw):
+    a = dict(state=A, codes=A, scales=A, n=2, H=4, d_k=128, d_v=128, qdq=2, stream=None)
+    a.update(kw)
+    if unpack:
+        return lib.gdn_state_unpack(a["codes"], a["scales"], a["state"], a["n"], a["H"],
+                                    a["d_k"], a["d_v"], a["qdq"], a["stream"])
+    return lib.gdn_state_pack(a["state"], a["codes"], a["scales"], a["n"], a["H"], a["d_k"],
+                              a["d_v"], a["qdq"], a["stream"])
+
+
+@pytest.mark.parametrize("call", [pf, dc, dp])
 def test_validation_errors(lib, call):
     assert call(lib, n_seq=-1) == INVALID
     assert call(lib, H=0) == INVALID
@@ -115,6 +139,26 @@ def test_prefill_specific_errors(lib):
 def test_decode_specific_errors(lib):
     assert dc(lib, state=None) == INVALID
     assert dc(lib, state=A + 4) == INVALID
+
+
+def test_packed_state_errors(lib):
+    assert dp(lib, qdq=0) == UNSUPPORTED          # packing needs a quantizing codec
+    assert dp(lib, codes=None) == INVALID
+    assert dp(lib, scales=None) == INVALID
+    assert dp(lib, codes=A + 2) == INVALID        # codes and scales: 4-byte aligned
+    assert dp(lib, scales=A + 1) == INVALID
+    for unpack in (False, True):
+        assert cv(lib, unpack, qdq=0) == UNSUPPORTED
+        assert cv(lib, unpack, qdq=9) == UNSUPPORTED
+        assert cv(lib, unpack, d_k=96) == UNSUPPORTED
+        assert cv(lib, unpack, d_v=32) == UNSUPPORTED
+        assert cv(lib, unpack, H=0) == INVALID
+        assert cv(lib, unpack, n=-1) == INVALID
+        assert cv(lib, unpack, state=None) == INVALID
+        assert cv(lib, unpack, state=A + 4) == INVALID  # fp32 state: 16-byte aligned
+        assert cv(lib, unpack, codes=A + 2) == INVALID
+        assert cv(lib, unpack, scales=None) == INVALID
+        assert cv(lib, unpack, n=0) == OK             # empty batch: no work, no launch
 
 
 def test_binding_refuses_missing_library(tmp_path, monkeypatch):
