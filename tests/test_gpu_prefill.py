@@ -263,3 +263,21 @@ def test_malformed_cu_seqlens_reported(cuda_lib):
     assert ei.value.status == 1
     # the error word is cleared by the read
     assert cuda_lib.gdn_last_error() == 0
+
+
+@pytest.mark.parametrize("n_seq", [40, 300])
+@pytest.mark.parametrize("dtype,dk", [("bf16", 128), ("f32", 64)])
+def test_packed_order_many_sequences(cuda_lib, n_seq, dtype, dk):
+    """Packed batches are processed longest first when they have at most 256
+    sequences (each CTA ranks the lengths) and in index order beyond; either
+    way every (sequence, head) lands in its own place.  Lengths repeat, so
+    the rank's tie-break by index is exercised."""
+    rng = np.random.default_rng(1000 + n_seq)
+    lengths = tuple(int(x) for x in rng.choice([1, 7, 64, 65, 130], size=n_seq))
+    case = gs.Case("many", n_seq=n_seq, H=2, d_k=dk, d_v=dk, lengths=lengths, dtype=dtype,
+                   qdq="none", state="normal", seed=93)
+    inp = gs.generate(case)
+    o, s = run_gpu(cuda_lib, inp, case)
+    o_ref, s_ref = oracle.prefill(inp, case)
+    assert rel_err(o, o_ref.reshape(o.shape)) <= TOL[dtype]
+    assert per_unit_rel_err(s, s_ref, axes=(-2, -1)) <= TOL[dtype]
