@@ -235,12 +235,12 @@ __device__ __forceinline__ StateRef state_ref(float *state, uint8_t *codes, floa
 // One 256-thread CTA per slab.  QK: kQdqNone / kQdqFp8Tile / kQdqInt8;
 // GROUP: INT8 group width (16/32/64); PACKED: the state is stored as codes +
 // scales (QK != kQdqNone).  k, q and the per-key decays sit in shared memory
-// so the state values are the only large register footprint: <= 80
-// registers give 3 CTAs per SM (96 KB of fp32 state loads in flight); the
-// packed kernel, which moves 3.5x fewer bytes per slab and is bound by its
-// arithmetic, runs 4 CTAs per SM (<= 64 registers).
+// so the state values are the only large register footprint: <= 64
+// registers give 4 CTAs per SM (128 KB of fp32 state loads in flight; a few
+// spilled bytes in some specialisations cost less than a fourth of the CTA
+// slots: 3 CTAs per SM measured 8 % slower on the serving workload).
 template <typename Tin, int DK, int DV, bool PER_KEY, int QK, int GROUP, bool PACKED>
-__global__ void __launch_bounds__(256, PACKED ? 4 : 3)
+__global__ void __launch_bounds__(256, 4)
 decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
               const Tin *__restrict__ v, const float *__restrict__ g,
               const float *__restrict__ beta, float *__restrict__ state,
