@@ -97,6 +97,15 @@ typedef enum {
  * The state QDQ runs after tokens 64, 128, ... of each sequence (counted from
  * its own start) and after its last token.
  *
+ * Kernel choice (results agree within the documented tolerances; they can
+ * differ in the last bits of o): bf16 GDN at d_k = d_v = 128 runs on the
+ * tensor cores, with either one CTA per (sequence, head) or a CTA pair (a
+ * thread-block cluster of two: one CTA computes each chunk's A, Aqk and
+ * triangular solve a chunk ahead, the other carries the state).  Pairs are
+ * used when every (sequence, head) gets its pair in one wave on the current
+ * device; the environment variable GDN_PREFILL_CTA_PAIR=0 or =1, read at
+ * every call, forces one CTA or the pair.
+ *
  * Returns GDN_OK after a successful launch (or when there is no work).
  */
 gdn_status gdn_prefill(const void *q, const void *k, const void *v,

@@ -13,7 +13,9 @@
 #include "gdn_common.cuh"
 #include "gdn_decode.cuh"
 #include "gdn_prefill_simt.cuh"
+#include "gdn_prefill_pair.cuh"
 #include "gdn_prefill_tc.cuh"
+#include <stdlib.h>
 
 namespace {
 
@@ -239,6 +241,64 @@ gdn_status launch_tc_one(const CUtensorMap &mq, const CUtensorMap &mk, const CUt
   return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
+// The same chunk algebra split over a CTA pair (one thread-block cluster of
+// two per (sequence, head)): the producer CTA computes A, Aqk and T a chunk
+// ahead, the chain CTA carries the state.
+template <int QK, int GR>
+gdn_status launch_pair_one(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                           const CUtensorMap &mo, const float *g, const float *beta,
+                           const float *state_in,
+                           const int32_t *cu, int T, int H, float scale, __nv_bfloat16 *o,
+                           float *state_out, unsigned *err, unsigned units, cudaStream_t st) {
+  auto kern = gdn::pair::prefill_pair_kernel<QK, GR>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)gdn::pair::kSmemBytes) != cudaSuccess)
+    return GDN_ERR_CUDA;
+  kern<<<2 * units, gdn::pair::kThreads, gdn::pair::kSmemBytes, st>>>(
+      mq, mk, mv, mo, g, beta, state_in, cu, T, H, scale, o, state_out, err);
+  return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+// How many CTA pairs of the tensor-core prefill can be resident at once on
+// the current device (0 if the pair kernel cannot run), cached per device.
+int g_pair_slots[kMaxDevices];
+bool g_pair_slots_known[kMaxDevices];
+
+int pair_slots() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  if (!g_pair_slots_known[dev]) {
+    auto kern = gdn::pair::prefill_pair_kernel<gdn::kQdqFp8Tile, 32>;
+    int n = 0;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)gdn::pair::kSmemBytes) == cudaSuccess) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(2, 1, 1);
+      cfg.blockDim = dim3(gdn::pair::kThreads, 1, 1);
+      cfg.dynamicSmemBytes = gdn::pair::kSmemBytes;
+      if (cudaOccupancyMaxActiveClusters(&n, (void *)kern, &cfg) != cudaSuccess) n = 0;
+    }
+    cudaGetLastError();  // a refused query leaves no sticky error behind
+    g_pair_slots[dev] = n;
+    g_pair_slots_known[dev] = true;
+  }
+  return g_pair_slots[dev];
+}
+
+// Schedule of the bf16 d = 128 GDN prefill.  A pair finishes a (sequence,
+// head) faster than one CTA but takes two SMs, so pairs pay when every unit
+// gets its pair at once (one wave); with more units than pair slots the
+// single-CTA kernel keeps more units in flight.  GDN_PREFILL_CTA_PAIR=1 or 0
+// in the environment forces the pair or the single-CTA kernel.
+bool use_pair(long long units) {
+  const char *e = getenv("GDN_PREFILL_CTA_PAIR");
+  if (e && e[0] == '0' && e[1] == 0) return false;
+  const int slots = pair_slots();
+  if (slots <= 0) return false;
+  if (e && e[0] == '1' && e[1] == 0) return true;
+  return units <= slots;
+}
+
 gdn_status launch_prefill_tc(const void *q, const void *k, const void *v, const float *g,
                              const float *beta, const float *state_in, const int32_t *cu,
                              int n_seq, int T, int H, int kind, int group, void *o,
@@ -256,6 +316,19 @@ gdn_status launch_prefill_tc(const void *q, const void *k, const void *v, const 
   const float scale = (float)(1.0 / sqrt(128.0));
   __nv_bfloat16 *oo = static_cast<__nv_bfloat16 *>(o);
   const unsigned nb = (unsigned)blocks;
+  if (use_pair(blocks)) {
+    if (blocks > 0x3fffffffLL) return GDN_ERR_UNSUPPORTED;
+    CUtensorMap mo;  // outputs [rows, H, 128] bf16, stored by whole 64-token chunks
+    if ((s = make_token_map(&mo, o, H, rows, false)) != GDN_OK) return s;
+#define GDN_TP(QK, GR) \
+  launch_pair_one<QK, GR>(mq, mk, mv, mo, g, beta, state_in, cu, T, H, scale, oo, state_out, err, nb, st)
+    if (kind == gdn::kQdqNone) return GDN_TP(gdn::kQdqNone, 32);
+    if (kind == gdn::kQdqFp8Tile) return GDN_TP(gdn::kQdqFp8Tile, 32);
+    if (group == 16) return GDN_TP(gdn::kQdqInt8, 16);
+    if (group == 64) return GDN_TP(gdn::kQdqInt8, 64);
+    return GDN_TP(gdn::kQdqInt8, 32);
+#undef GDN_TP
+  }
 #define GDN_TC(QK, GR) \
   launch_tc_one<QK, GR>(mq, mk, mv, g, beta, state_in, cu, T, H, scale, oo, state_out, err, nb, st)
   if (kind == gdn::kQdqNone) return GDN_TC(gdn::kQdqNone, 32);

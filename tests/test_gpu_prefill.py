@@ -13,6 +13,9 @@
   configuration compared on sampled (sequence, head) units;
 * edge cases: empty sequences, an all-empty packed batch, a malformed
   cu_seqlens reported through gdn_last_error, state_out aliasing state_in.
+
+Every test runs three times: under the automatic schedule choice and with
+the single-CTA and the CTA-pair tensor-core kernels forced.
 """
 
 import numpy as np
@@ -24,6 +27,19 @@ import oracle
 from parity import TOL, assert_flip_budget, check_codes, per_unit_rel_err, rel_err
 
 pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True, params=["auto", "single", "pair"])
+def schedule(request, monkeypatch):
+    """Every case under the library's own choice of tensor-core schedule and
+    under each schedule forced (GDN_PREFILL_CTA_PAIR): one CTA per
+    (sequence, head), or a CTA pair.  Cases off the tensor-core path (fp32,
+    KDA gates, d = 64) run the same kernel in all three."""
+    if request.param == "auto":
+        monkeypatch.delenv("GDN_PREFILL_CTA_PAIR", raising=False)
+    else:
+        monkeypatch.setenv("GDN_PREFILL_CTA_PAIR", "1" if request.param == "pair" else "0")
+    return request.param
 
 
 def dev(x):
