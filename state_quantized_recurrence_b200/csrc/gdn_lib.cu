@@ -319,7 +319,7 @@ gdn_status launch_prefill_tc(const void *q, const void *k, const void *v, const 
   if (use_pair(blocks)) {
     if (blocks > 0x3fffffffLL) return GDN_ERR_UNSUPPORTED;
     CUtensorMap mo;  // outputs [rows, H, 128] bf16, stored by whole 64-token chunks
-    if ((s = make_token_map(&mo, o, H, rows, false)) != GDN_OK) return s;
+    if ((s = make_token_map(&mo, o, H, rows, true)) != GDN_OK) return s;
 #define GDN_TP(QK, GR) \
   launch_pair_one<QK, GR>(mq, mk, mv, mo, g, beta, state_in, cu, T, H, scale, oo, state_out, err, nb, st)
     if (kind == gdn::kQdqNone) return GDN_TP(gdn::kQdqNone, 32);

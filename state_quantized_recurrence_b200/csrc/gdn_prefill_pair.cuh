@@ -579,23 +579,47 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     auto out_epilogue = [&](int j, long long tbj, int nj, float hs_j) {
       const Gates *gj = &sm->gt[j % 3];
       const uint32_t reg = (uint32_t)(j & 1) * TM_REG;
-      float qh[32], av[32];
-      sm100::tmem_ld32(tmem + lane_off + reg + TM_QH + 32 * wg, qh);
-      sm100::tmem_ld32(tmem + lane_off + reg + 32 * wg, av);
       const float sh = scale * hs_j;
-#pragma unroll
-      for (int t = 0; t < 32; t += 4) {
-        const float4 g4 = *reinterpret_cast<const float4 *>(gj->gam + 32 * wg + t);
-        qh[t] = fmaf(sh * g4.x, qh[t], scale * av[t]);
-        qh[t + 1] = fmaf(sh * g4.y, qh[t + 1], scale * av[t + 1]);
-        qh[t + 2] = fmaf(sh * g4.z, qh[t + 2], scale * av[t + 2]);
-        qh[t + 3] = fmaf(sh * g4.w, qh[t + 3], scale * av[t + 3]);
-      }
       if (nj == kC) {
-        __nv_bfloat16 *tile = reinterpret_cast<__nv_bfloat16 *>(gbase + C_O + (row >> 6) * 8192) +
-                              32 * wg * 64 + (row & 63);
+        // Fragments of 16 value rows x 32 tokens (two per warp), combined,
+        // packed to bf16 token pairs and stored transposed into the tile
+        // [v half][t][64 v] (128-byte rows, 16-byte chunks swizzled by t % 8).
+        const int c = lane & 3, gq = lane >> 2;
 #pragma unroll
-        for (int t = 0; t < 32; ++t) tile[t * 64] = __float2bfloat16_rn(qh[t]);
+        for (int hl = 0; hl < 2; ++hl) {
+          const int L = 32 * (warp & 3) + 16 * hl;  // first value row of the block
+          const uint32_t lsel = (uint32_t)L << 16;
+          uint32_t qh[16], av[16];
+          sm100::tmem_ld16x256b_x4(tmem + lsel + reg + TM_QH + 32 * wg, qh);
+          sm100::tmem_ld16x256b_x4(tmem + lsel + reg + 32 * wg, av);
+          uint32_t pk[8];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 g2 = *reinterpret_cast<const float2 *>(gj->gam + 32 * wg + 8 * k + 2 * c);
+            const float s0 = sh * g2.x, s1 = sh * g2.y;
+#pragma unroll
+            for (int hv = 0; hv < 2; ++hv) {  // value rows L + gq and L + 8 + gq
+              const int e = 4 * k + 2 * hv;
+              const float o0 = fmaf(s0, __uint_as_float(qh[e]), scale * __uint_as_float(av[e]));
+              const float o1 = fmaf(s1, __uint_as_float(qh[e + 1]), scale * __uint_as_float(av[e + 1]));
+              __nv_bfloat162 p2 = __floats2bfloat162_rn(o0, o1);
+              pk[2 * k + hv] = *reinterpret_cast<uint32_t *>(&p2);
+            }
+          }
+          // matrix m of an instruction: tokens 32 wg + 8 (k0 + m / 2) .. + 7,
+          // values L + 8 (m % 2) .. + 7; this thread addresses row lane % 8 of
+          // matrix lane / 8
+#pragma unroll
+          for (int k0 = 0; k0 < 4; k0 += 2) {
+            const int m = lane >> 3, rr = lane & 7;
+            const int t = 32 * wg + 8 * (k0 + (m >> 1)) + rr;
+            const int v0 = L + 8 * (m & 1);
+            const uint32_t addr = base + C_O + (uint32_t)(v0 >> 6) * 8192u + (uint32_t)t * 128u +
+                                  ((uint32_t)(((v0 & 63) >> 3) ^ (t & 7)) << 4);
+            sm100::stmatrix_x4_trans(addr, pk[2 * k0], pk[2 * k0 + 1], pk[2 * k0 + 2],
+                                     pk[2 * k0 + 3]);
+          }
+        }
         sm100::fence_proxy_async();
         asm volatile("bar.sync 5, 256;" ::: "memory");
         if (tid == kStoreTid) {
@@ -604,12 +628,17 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           sm100::bulk_commit();
         }
       } else {
+        float qh[32], av[32];
+        sm100::tmem_ld32(tmem + lane_off + reg + TM_QH + 32 * wg, qh);
+        sm100::tmem_ld32(tmem + lane_off + reg + 32 * wg, av);
         const int cnt = nj - 32 * wg;
         __nv_bfloat16 *dst = o + ((tbj + 32 * wg) * H + h) * kD + row;
         const long long ts = (long long)H * kD;
 #pragma unroll
-        for (int t = 0; t < 32; ++t)
-          if (t < cnt) dst[t * ts] = __float2bfloat16_rn(qh[t]);
+        for (int t = 0; t < 32; ++t) {
+          const float ot = fmaf(sh * gj->gam[32 * wg + t], qh[t], scale * av[t]);
+          if (t < cnt) dst[t * ts] = __float2bfloat16_rn(ot);
+        }
       }
     };
 
@@ -857,8 +886,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             for (int i = 0; i < 32; i += 4)
               *reinterpret_cast<float4 *>(dst + i) = make_float4(y[i], y[i + 1], y[i + 2], y[i + 3]);
           } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) y[i] *= gn_next;
+            scale32(y, gn_next);
             sm100::tmem_st32(tmem + lane_off + TM_D4 + c0v, y);
           }
         }

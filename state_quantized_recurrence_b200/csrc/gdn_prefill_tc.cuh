@@ -736,8 +736,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           for (int i = 0; i < 32; i += 4)
             *reinterpret_cast<float4 *>(dst + i) = make_float4(y[i], y[i + 1], y[i + 2], y[i + 3]);
         } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) y[i] *= gn_next;
+          scale32(y, gn_next);
           sm100::tmem_st32(tmem + lane_off + TM_D4 + c0v, y);
         }
       }

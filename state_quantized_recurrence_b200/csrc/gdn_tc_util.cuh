@@ -63,23 +63,51 @@ __device__ __forceinline__ void store32_hl(uint32_t thi, uint32_t tlo, int r, in
   }
 }
 
+// Packed fp32 pairs (sm_100 f32x2 arithmetic: each lane rounds exactly as
+// the scalar instruction, two lanes per instruction).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+  return d;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float &lo, float &hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+// y[i] *= s for 32 values.
+__device__ __forceinline__ void scale32(float *y, float s) {
+  const uint64_t s2 = f2_pack(s, s);
+#pragma unroll
+  for (int i = 0; i < 32; i += 2) f2_unpack(f2_mul(f2_pack(y[i], y[i + 1]), s2), y[i], y[i + 1]);
+}
+
 // E4M3 codes of x0/s2 and x1/s2 (correctly rounded quotients from r = RN(1/s2),
 // Markstein's correction), returned as an fp16 pair (exact); y0, y1 receive
 // the dequantized values code * s (s = s2 unless the operands were
 // pre-scaled by a power of two).
 __device__ __forceinline__ uint32_t fp8_code_pair(float x0, float x1, float s2, float r, float &y0,
                                                   float &y1, float s = 0.0f) {
-  const float q0 = __fmul_rn(x0, r), q1 = __fmul_rn(x1, r);
-  const float t0 = __fmaf_rn(__fmaf_rn(-q0, s2, x0), r, q0);
-  const float t1 = __fmaf_rn(__fmaf_rn(-q1, s2, x1), r, q1);
+  const uint64_t x = f2_pack(x0, x1), rr = f2_pack(r, r);
+  const uint64_t q = f2_mul(x, rr);
+  const uint64_t t = f2_fma(f2_fma(q, f2_pack(-s2, -s2), x), rr, q);
+  float t0, t1;
+  f2_unpack(t, t0, t1);
   const __nv_fp8x2_storage_t f8 =
       __nv_cvt_float2_to_fp8x2(make_float2(t0, t1), __NV_SATFINITE, __NV_E4M3);
   const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(f8, __NV_E4M3);
   const __half2 hh = *reinterpret_cast<const __half2 *>(&hr);
   const float2 cf = __half22float2(hh);
   const float sd = s == 0.0f ? s2 : s;
-  y0 = __fmul_rn(cf.x, sd);
-  y1 = __fmul_rn(cf.y, sd);
+  f2_unpack(f2_mul(f2_pack(cf.x, cf.y), f2_pack(sd, sd)), y0, y1);
   return *reinterpret_cast<const uint32_t *>(&hh);
 }
 
