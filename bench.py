@@ -282,14 +282,17 @@ def measure_prefill(args, dist, dev, stream, sampler, peaks, case, steps, warmup
     flops = prefill_flops(tokens, case.H, case.d_k, case.d_v)
     gbs = nbytes / (ms / 1e3) / 1e9
     tfs = flops / (ms / 1e3) / 1e12
-    tc = case.dtype == "bf16" and case.gate == "scalar" and case.d_k == 128 and case.d_v == 128
+    kernel = {"tc_cta_pair": "pair::prefill_pair_kernel (tcgen05, CTA pair per unit)",
+              "tc_one_cta": "tc::prefill_tc_kernel (tcgen05, one CTA per unit)",
+              "cuda_cores": "simt::prefill_simt_kernel (FFMA)"}[
+        sqr.gdn_prefill_schedule(case.n_seq, case.H, case.d_k, case.d_v, d["q"].dtype, case.gate)]
     res = {
         "workload": f"{case.name}: n_seq={case.n_seq} H={case.H} tokens={tokens} d={case.d_k}, "
                     f"{case.dtype}, {case.gate} gate, {case.qdq}, "
                     f"{'random' if inp['state_in'] is not None else 'zero'} initial state",
         "value": round(dist.world * tokens / (ms_max / 1e3), 1), "unit": "tokens/s",
         "ms_per_step": round(ms_max, 5), "steps": steps,
-        "kernel": "tc::prefill_tc_kernel (tcgen05)" if tc else "simt::prefill_simt_kernel (FFMA)",
+        "kernel": kernel,
         "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
                      "traffic": (None if (args.small or traffic_key is None)
@@ -335,7 +338,7 @@ def run_ours(args, dist: Dist) -> dict:
         case = gs.small_case("gdn_prefill", T=512)
     head, (inp, d, o, st, step, tokens, nbytes) = measure_prefill(
         args, dist, dev, stream, sampler, peaks, case, args.steps, args.warmup,
-        traffic_key="prefill_tc", keep=True)
+        traffic_key="prefill_gdn", keep=True)
     ms_max = head["ms_per_step"]
     value = head["value"]
     clocks = head["clocks"]

@@ -28,7 +28,7 @@ def _load() -> ctypes.CDLL:
     if not os.path.exists(library_path):
         raise ImportError(
             f"CUDA library {library_path} is missing; build it with "
-            "`python -m state_quantized_recurrence_b200.build` (there is no fallback)")
+            "`python state_quantized_recurrence_b200/build.py` (there is no fallback)")
     L = ctypes.CDLL(library_path)
     P, I = ctypes.c_void_p, ctypes.c_int
     L.gdn_prefill.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P, P, P]
@@ -47,6 +47,8 @@ def _load() -> ctypes.CDLL:
     L.gdn_status_string.restype = ctypes.c_char_p
     L.gdn_version.argtypes = []
     L.gdn_version.restype = I
+    L.gdn_prefill_schedule.argtypes = [I, I, I, I, I, I]
+    L.gdn_prefill_schedule.restype = I
     return L
 
 
@@ -72,6 +74,20 @@ def _check_dev(*ts):
     for t in ts:
         if t is not None:
             _need(t.is_cuda and t.is_contiguous(), "tensors must be contiguous CUDA tensors")
+
+
+GDN_PREFILL_KERNEL = {0: "cuda_cores", 1: "tc_one_cta", 2: "tc_cta_pair"}
+
+
+def gdn_prefill_schedule(n_seq: int, H: int, d_k: int, d_v: int, dtype=torch.bfloat16,
+                         gate: str = "scalar") -> str:
+    """Which prefill kernel gdn_prefill launches for these shapes on the
+    current device: "cuda_cores", "tc_one_cta" or "tc_cta_pair"."""
+    _need(dtype in GDN_DTYPE and gate in GDN_GATE, "unsupported dtype or gate kind")
+    r = int(lib.gdn_prefill_schedule(int(n_seq), int(H), int(d_k), int(d_v), GDN_DTYPE[dtype],
+                                     GDN_GATE[gate]))
+    _need(r >= 0, "shapes gdn_prefill does not support")
+    return GDN_PREFILL_KERNEL[r]
 
 
 def gdn_last_error(stream=None) -> int:

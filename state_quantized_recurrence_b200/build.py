@@ -1,6 +1,6 @@
 """Build the CUDA library ``libgdn_qdq.so`` in-tree for sm_100a.
 
-    python -m state_quantized_recurrence_b200.build [--force]
+    python state_quantized_recurrence_b200/build.py [--force]
 
 nvcc cross-compiles without a GPU.  The shared library sits next to this
 file so that it travels with the source tree.

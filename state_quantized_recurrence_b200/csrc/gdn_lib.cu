@@ -299,6 +299,13 @@ bool use_pair(long long units) {
   return units <= slots;
 }
 
+// bf16 GDN at d_k = d_v = 128 runs on the tensor cores; fp32 inputs (whose
+// 1e-5 tolerance the fp16 operand splits cannot promise), per-key (KDA)
+// gates and d = 64 run on the CUDA-core kernel.
+bool tc_path(gdn_dtype dt, gdn_gate_kind gk, int d_k, int d_v) {
+  return dt == GDN_DTYPE_BF16 && gk == GDN_GATE_SCALAR && d_k == 128 && d_v == 128;
+}
+
 gdn_status launch_prefill_tc(const void *q, const void *k, const void *v, const float *g,
                              const float *beta, const float *state_in, const int32_t *cu,
                              int n_seq, int T, int H, int kind, int group, void *o,
@@ -446,7 +453,7 @@ gdn_status gdn_prefill(const void *q, const void *k, const void *v, const float 
   // tensor cores; fp32 inputs (whose 1e-5 tolerance the fp16 operand splits
   // cannot promise), per-key (KDA) gates and d = 64 run on the CUDA-core
   // kernel.  Both compute the same chunked algebra.
-  if (dt == GDN_DTYPE_BF16 && !pk && d_k == 128 && d_v == 128)
+  if (tc_path(dt, gk, d_k, d_v))
     return launch_prefill_tc(q, k, v, g, beta, state_in, cu_seqlens, n_seq, T, H, kind, group, o,
                              state_out, err, st);
   if (dt == GDN_DTYPE_BF16)
@@ -454,6 +461,16 @@ gdn_status gdn_prefill(const void *q, const void *k, const void *v, const float 
                                               H, d_k, d_v, pk, kind, group, o, state_out, err, st);
   return launch_prefill_simt<float>(q, k, v, g, beta, state_in, cu_seqlens, n_seq, T, H, d_k,
                                     d_v, pk, kind, group, o, state_out, err, st);
+}
+
+int gdn_prefill_schedule(int n_seq, int H, int d_k, int d_v, gdn_dtype dt, gdn_gate_kind gk) {
+  if (n_seq < 0 || H <= 0) return -1;
+  if ((d_k != 64 && d_k != 128) || (d_v != 64 && d_v != 128)) return -1;
+  if (dt != GDN_DTYPE_BF16 && dt != GDN_DTYPE_F32) return -1;
+  if (gk != GDN_GATE_SCALAR && gk != GDN_GATE_PER_KEY) return -1;
+  if (!tc_path(dt, gk, d_k, d_v)) return GDN_PREFILL_CUDA_CORES;
+  const long long units = (long long)n_seq * H;
+  return use_pair(units) ? GDN_PREFILL_TC_CTA_PAIR : GDN_PREFILL_TC_ONE_CTA;
 }
 
 gdn_status gdn_last_error(void *cuda_stream) {

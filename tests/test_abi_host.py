@@ -25,7 +25,12 @@ BF16, F32 = 0, 1
 
 @pytest.fixture(scope="module")
 def lib():
-    from state_quantized_recurrence_b200 import build
+    import importlib.util  # the build script by path: the package import needs the library
+    spec = importlib.util.spec_from_file_location(
+        "state_quantized_recurrence_b200_build",
+        os.path.join(ROOT, "state_quantized_recurrence_b200", "build.py"))
+    build = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(build)
     build.build()
     L = ctypes.CDLL(LIB)
     P, I = ctypes.c_void_p, ctypes.c_int
@@ -169,3 +174,17 @@ def test_binding_refuses_missing_library(tmp_path, monkeypatch):
     with pytest.raises(ImportError):
         b._load()
     importlib.reload(b)
+
+
+def test_prefill_schedule_host_cases(lib):
+    """Shapes off the tensor-core path choose the CUDA-core kernel without
+    touching a device; shapes gdn_prefill rejects give -1."""
+    I = ctypes.c_int
+    lib.gdn_prefill_schedule.argtypes = [I] * 6
+    lib.gdn_prefill_schedule.restype = I
+    assert lib.gdn_prefill_schedule(2, 4, 128, 128, 1, 0) == 0   # fp32
+    assert lib.gdn_prefill_schedule(2, 4, 128, 128, 0, 1) == 0   # KDA gates
+    assert lib.gdn_prefill_schedule(2, 4, 64, 64, 0, 0) == 0     # d = 64
+    assert lib.gdn_prefill_schedule(2, 4, 96, 128, 0, 0) == -1
+    assert lib.gdn_prefill_schedule(2, 0, 128, 128, 0, 0) == -1
+    assert lib.gdn_prefill_schedule(2, 4, 128, 128, 7, 0) == -1

@@ -297,3 +297,19 @@ def test_packed_order_many_sequences(cuda_lib, n_seq, dtype, dk):
     o_ref, s_ref = oracle.prefill(inp, case)
     assert rel_err(o, o_ref.reshape(o.shape)) <= TOL[dtype]
     assert per_unit_rel_err(s, s_ref, axes=(-2, -1)) <= TOL[dtype]
+
+
+def test_schedule_is_the_one_forced(cuda_lib, schedule):
+    """The forced schedules are the ones launched; the automatic choice takes
+    the pair while every unit gets one in a wave, one CTA per unit beyond."""
+    pick = cuda_lib.gdn_prefill_schedule
+    if schedule == "pair":
+        assert pick(4, 16, 128, 128) == "tc_cta_pair"
+    elif schedule == "single":
+        assert pick(4, 16, 128, 128) == "tc_one_cta"
+    else:
+        assert pick(4, 16, 128, 128) == "tc_cta_pair"
+        assert pick(64, 16, 128, 128) == "tc_one_cta"
+    assert pick(4, 16, 128, 128, dtype=torch.float32) == "cuda_cores"
+    assert pick(4, 16, 128, 128, gate="per_key") == "cuda_cores"
+
