@@ -50,12 +50,20 @@ def load_peaks() -> dict:
         return dict(FALLBACK_PEAKS)
 
 
-def kernel_source_hash() -> str:
-    """Hash of the CUDA sources; recorded DRAM traffic is valid only for it."""
-    import glob
+# The CUDA sources each recorded kernel is compiled from (its launch
+# configuration in gdn_lib.cu is fixed per workload).
+KERNEL_SOURCES = {
+    "prefill_gdn": ["gdn_prefill_pair.cuh", "gdn_tc_util.cuh", "gdn_sm100.cuh", "gdn_common.cuh"],
+    "decode": ["gdn_decode.cuh", "gdn_common.cuh"],
+    "decode_packed": ["gdn_decode.cuh", "gdn_common.cuh"],
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
+    """Hash of `kernel`'s CUDA sources; its recorded DRAM traffic is valid only for it."""
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "state_quantized_recurrence_b200", "csrc", "*"))):
-        h.update(open(f, "rb").read())
+    for f in KERNEL_SOURCES[kernel]:
+        h.update(open(os.path.join(ROOT, "state_quantized_recurrence_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
 
@@ -66,7 +74,8 @@ def recorded_traffic(kernel: str):
         rec = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))[kernel]
     except (OSError, ValueError, KeyError):
         return None
-    return rec.get("bytes_per_launch") if rec.get("source_hash") == kernel_source_hash() else None
+    ok = rec.get("source_hash") == kernel_source_hash(kernel)
+    return rec.get("bytes_per_launch") if ok else None
 
 
 # ------------------------------------------------------------ workload math
@@ -325,8 +334,8 @@ def run_ours(args, dist: Dist) -> dict:
     stream = torch.cuda.current_stream(dev)
     sampler = ClockSampler(dist.local)
 
-    if args.only == "decode":  # profiler captures of the decode kernel alone
-        dec = run_decode(args, dist, dev, stream, sampler, peaks)
+    if args.only in ("decode", "decode_packed"):  # profiler captures of one decode kernel
+        dec = run_decode(args, dist, dev, stream, sampler, peaks, packed=args.only == "decode_packed")
         sampler.stop()
         dist.close()
         return {"metric": dec["metric"], "value": dec["value"], "unit": dec["unit"],
@@ -563,7 +572,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-decode", action="store_true")
-    ap.add_argument("--only", choices=["prefill", "decode"], default=None,
+    ap.add_argument("--only", choices=["prefill", "decode", "decode_packed"], default=None,
                     help="measure one kernel only (profiler captures)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-others", action="store_true",
