@@ -178,6 +178,55 @@ def test_solve_identities_64():
     assert np.abs(chunked.neumann_inverse(A, 3) - T).max() > 1e-6
 
 
+@pytest.mark.parametrize("degree", [1, 3, 7, 15, 31])
+def test_neumann_residual_identity(degree):
+    """(I + A) sum_{n<=d} (-A)^n = I - (-A)^(d+1): a dropped or extra term, a
+    sign slip or an off-by-one degree breaks it.  The right side comes from
+    numpy's matrix power, not from the oracle's series."""
+    rng = np.random.default_rng(40 + degree)
+    A = np.tril(rng.standard_normal((64, 64)) * 0.15, -1)
+    Td = chunked.neumann_inverse(A, degree)
+    rhs = np.eye(64) - np.linalg.matrix_power(-A, degree + 1)
+    np.testing.assert_allclose((np.eye(64) + A) @ Td, rhs, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("m", [1, 2, 3, 4, 5, 6])
+def test_neumann_product_form(m):
+    """For degree 2^m - 1 the series factors as prod_{i<m} (I + X^(2^i)),
+    X = -A (the GPU evaluates this form)."""
+    rng = np.random.default_rng(60 + m)
+    A = np.tril(rng.standard_normal((64, 64)) * 0.15, -1)
+    X = -A
+    P = np.eye(64)
+    for i in range(m):
+        P = P @ (np.eye(64) + np.linalg.matrix_power(X, 2 ** i))
+    np.testing.assert_allclose(chunked.neumann_inverse(A, 2 ** m - 1), P, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("degree", [3, 7])
+def test_neumann_exact_on_short_chunks(degree):
+    """A chunk of n tokens has an n x n strictly lower A, so A^n = 0: the
+    degree-d series is the exact inverse whenever n <= d + 1.  Sequences of
+    n <= d + 1 tokens give the exact chunked result (and the token
+    recurrence); a full 64-token chunk does not."""
+    rng = np.random.default_rng(70 + degree)
+    lengths = [1, degree, degree + 1, 64]
+    T, H, dk, dv = sum(lengths), 2, 32, 16
+    q, k, v, g, beta = _rand(rng, T, H, dk, dv, True)
+    H0 = rng.standard_normal((len(lengths), H, dk, dv)) * 0.05
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int64)
+    o_e, s_e = chunked.chunked_wy(q, k, v, g, beta, H0, cu, per_key_gate=True)
+    o_n, s_n = chunked.chunked_wy(q, k, v, g, beta, H0, cu, per_key_gate=True,
+                                  solve=("neumann", degree))
+    o_r, _ = _run(q, k, v, g, beta, H0, lengths, True)
+    np.testing.assert_allclose(o_e, o_r, rtol=0, atol=1e-12)
+    short = slice(0, int(cu[3]))
+    np.testing.assert_allclose(o_n[short], o_e[short], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(s_n[:3], s_e[:3], rtol=0, atol=1e-12)
+    assert np.abs(o_n[int(cu[3]):] - o_e[int(cu[3]):]).max() > 1e-9
+    assert np.abs(s_n[3] - s_e[3]).max() > 1e-9
+
+
 @pytest.mark.parametrize("mode", ["int8_g32", "fp8_tile64"])
 def test_qdq_placement_prefill(mode):
     rng = np.random.default_rng(18)
