@@ -178,6 +178,27 @@ gdn_status gdn_decode_packed(const void *q, const void *k, const void *v,
 gdn_status gdn_last_error(void *cuda_stream);
 
 /*
+ * gdn_prefill_neumann - gdn_prefill with the approximate triangular solve of
+ * the approximate-inverse PR (#2507, What section: an explicit Neumann
+ * polynomial degree, no silent change of degree, no fallback): every chunk's
+ * (I + A)^-1 is replaced by T_d = sum_{n=0}^{d} (-A)^n, evaluated as
+ * prod_{i<m} (I + (-A)^(2^i)) for d = 2^m - 1.
+ *
+ * degree: one of 1, 3, 7, 15, 31, 63, else GDN_ERR_INVALID_ARG (nothing is
+ *   launched).  A chunk of n tokens has A^n = 0, so degree >= n - 1 gives
+ *   the exact solve for it; 63 is exact for every chunk.
+ * All other arguments, layouts, ownership and errors as gdn_prefill.  Runs
+ * on the CUDA-core (FFMA) kernel for every dtype, gate kind and shape.
+ */
+gdn_status gdn_prefill_neumann(const void *q, const void *k, const void *v,
+                               const float *g, const float *beta,
+                               const float *state_in, const int32_t *cu_seqlens,
+                               int n_seq, int T, int H, int d_k, int d_v,
+                               gdn_dtype dt, gdn_gate_kind gk, gdn_qdq_mode qdq,
+                               int degree, void *o, float *state_out,
+                               void *cuda_stream);
+
+/*
  * gdn_prefill_schedule - which prefill kernel gdn_prefill launches for these
  * shapes on the current device, under the current GDN_PREFILL_CTA_PAIR
  * setting (the same selection code).  Host-only; it may query the device's

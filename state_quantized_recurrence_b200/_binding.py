@@ -33,6 +33,8 @@ def _load() -> ctypes.CDLL:
     P, I = ctypes.c_void_p, ctypes.c_int
     L.gdn_prefill.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P, P, P]
     L.gdn_prefill.restype = I
+    L.gdn_prefill_neumann.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, P, P, P]
+    L.gdn_prefill_neumann.restype = I
     L.gdn_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, P, P]
     L.gdn_decode.restype = I
     L.gdn_decode_packed.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, P]
@@ -106,12 +108,15 @@ def _gate_kind(g: torch.Tensor, lead: int) -> str:
 
 
 def gdn_prefill_into(q, k, v, g, beta, state_in, cu_seqlens, o, state_out,
-                     qdq: str = "fp8_tile64", stream=None) -> None:
+                     qdq: str = "fp8_tile64", stream=None,
+                     neumann_degree: Optional[int] = None) -> None:
     """Chunked prefix writing into preallocated ``o`` and ``state_out``.
 
     Dense: q, k [B, T, H, d_k], v/o [B, T, H, d_v]; packed (cu_seqlens int32
     [n_seq + 1]): [1, T_total, H, d].  g: fp32 [.., H] or [.., H, d_k];
-    beta fp32 [.., H]; states fp32 [n_seq, H, d_k, d_v].
+    beta fp32 [.., H]; states fp32 [n_seq, H, d_k, d_v].  ``neumann_degree``
+    (1, 3, 7, 15, 31 or 63) selects the approximate solve
+    (gdn_prefill_neumann); None the exact one.
     """
     _check_dev(q, k, v, g, beta, state_in, cu_seqlens, o, state_out)
     _need(q.dim() == 4 and k.shape == q.shape and v.dim() == 4, "q, k, v must be [B, T, H, d]")
@@ -135,21 +140,26 @@ def gdn_prefill_into(q, k, v, g, beta, state_in, cu_seqlens, o, state_out,
     if state_in is not None:
         _need(state_in.shape == state_out.shape and state_in.dtype == torch.float32,
               "state_in must be fp32 [n_seq, H, d_k, d_v]")
-    s = lib.gdn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_in),
-                        _ptr(cu_seqlens), n_seq, T_arg, H, d_k, d_v, GDN_DTYPE[q.dtype],
-                        GDN_GATE[gk], GDN_QDQ[qdq], _ptr(o), _ptr(state_out), _stream(stream))
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_in), _ptr(cu_seqlens),
+            n_seq, T_arg, H, d_k, d_v, GDN_DTYPE[q.dtype], GDN_GATE[gk], GDN_QDQ[qdq])
+    tail = (_ptr(o), _ptr(state_out), _stream(stream))
+    if neumann_degree is None:
+        s, where = lib.gdn_prefill(*args, *tail), "gdn_prefill"
+    else:
+        s, where = lib.gdn_prefill_neumann(*args, int(neumann_degree), *tail), "gdn_prefill_neumann"
     if s != 0:
-        raise GdnError(s, "gdn_prefill")
+        raise GdnError(s, where)
 
 
 def gdn_prefill(q, k, v, g, beta, state_in=None, cu_seqlens=None, qdq: str = "fp8_tile64",
-                stream=None):
+                stream=None, neumann_degree: Optional[int] = None):
     """Chunked prefix; returns ``(o, state_out)`` (allocated with torch)."""
     n_seq = q.shape[0] if cu_seqlens is None else cu_seqlens.numel() - 1
     o = torch.empty(v.shape, dtype=q.dtype, device=q.device)
     state_out = torch.empty((n_seq, q.shape[2], q.shape[3], v.shape[3]), dtype=torch.float32,
                             device=q.device)
-    gdn_prefill_into(q, k, v, g, beta, state_in, cu_seqlens, o, state_out, qdq, stream)
+    gdn_prefill_into(q, k, v, g, beta, state_in, cu_seqlens, o, state_out, qdq, stream,
+                     neumann_degree)
     return o, state_out
 
 

@@ -134,19 +134,35 @@ gdn_status launch_decode(const void *q, const void *k, const void *v, const floa
   return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
-template <typename Tin, int DK, bool PK>
-gdn_status launch_simt_one(const Tin *q, const Tin *k, const Tin *v, const float *g,
+template <typename Tin, int DK, bool PK, bool NEU>
+gdn_status launch_simt_neu(const Tin *q, const Tin *k, const Tin *v, const float *g,
                            const float *beta, const float *state_in, const int32_t *cu,
                            int T, int H, int d_v, float scale, int kind, int group, Tin *o,
-                           float *state_out, unsigned *err, unsigned blocks, cudaStream_t st) {
-  using L = gdn::simt::Smem<DK>;
-  auto kern = gdn::simt::prefill_simt_kernel<Tin, DK, PK>;
+                           float *state_out, unsigned *err, unsigned blocks, int neu_m,
+                           cudaStream_t st) {
+  using L = gdn::simt::Smem<DK, NEU>;
+  auto kern = gdn::simt::prefill_simt_kernel<Tin, DK, PK, NEU>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kBytes) !=
       cudaSuccess)
     return GDN_ERR_CUDA;
   kern<<<blocks, gdn::simt::kThreads, L::kBytes, st>>>(q, k, v, g, beta, state_in, cu, T, H, d_v,
-                                                       scale, kind, group, o, state_out, err);
+                                                       scale, kind, group, o, state_out, err,
+                                                       neu_m);
   return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+// neu_m = 0: exact solve; neu_m >= 1: Neumann degree 2^neu_m - 1.
+template <typename Tin, int DK, bool PK>
+gdn_status launch_simt_one(const Tin *q, const Tin *k, const Tin *v, const float *g,
+                           const float *beta, const float *state_in, const int32_t *cu,
+                           int T, int H, int d_v, float scale, int kind, int group, Tin *o,
+                           float *state_out, unsigned *err, unsigned blocks, int neu_m,
+                           cudaStream_t st) {
+  if (neu_m > 0)
+    return launch_simt_neu<Tin, DK, PK, true>(q, k, v, g, beta, state_in, cu, T, H, d_v, scale,
+                                              kind, group, o, state_out, err, blocks, neu_m, st);
+  return launch_simt_neu<Tin, DK, PK, false>(q, k, v, g, beta, state_in, cu, T, H, d_v, scale,
+                                             kind, group, o, state_out, err, blocks, 0, st);
 }
 
 template <int DK, int DV, bool TO>
@@ -179,7 +195,7 @@ gdn_status launch_prefill_simt(const void *q, const void *k, const void *v, cons
                                const float *beta, const float *state_in, const int32_t *cu,
                                int n_seq, int T, int H, int d_k, int d_v, bool per_key,
                                int kind, int group, void *o, float *state_out, unsigned *err,
-                               cudaStream_t st) {
+                               int neu_m, cudaStream_t st) {
   const long long blocks = (long long)n_seq * H * (d_v / 64);
   if (blocks > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
   const float scale = (float)(1.0 / sqrt((double)d_k));
@@ -188,7 +204,7 @@ gdn_status launch_prefill_simt(const void *q, const void *k, const void *v, cons
   Tin *oo = static_cast<Tin *>(o);
   const unsigned nb = (unsigned)blocks;
 #define GDN_PF(DK, PK) \
-  launch_simt_one<Tin, DK, PK>(qq, kk, vv, g, beta, state_in, cu, T, H, d_v, scale, kind, group, oo, state_out, err, nb, st)
+  launch_simt_one<Tin, DK, PK>(qq, kk, vv, g, beta, state_in, cu, T, H, d_v, scale, kind, group, oo, state_out, err, nb, neu_m, st)
   if (d_k == 128) return per_key ? GDN_PF(128, true) : GDN_PF(128, false);
   return per_key ? GDN_PF(64, true) : GDN_PF(64, false);
 #undef GDN_PF
@@ -346,6 +362,42 @@ gdn_status launch_prefill_tc(const void *q, const void *k, const void *v, const 
 #undef GDN_TC
 }
 
+// Validation and kernel choice shared by gdn_prefill and gdn_prefill_neumann
+// (neu_m = 0: exact solve; >= 1: Neumann degree 2^neu_m - 1).
+gdn_status prefill_impl(const void *q, const void *k, const void *v, const float *g,
+                        const float *beta, const float *state_in, const int32_t *cu_seqlens,
+                        int n_seq, int T, int H, int d_k, int d_v, gdn_dtype dt,
+                        gdn_gate_kind gk, gdn_qdq_mode qdq, int neu_m, void *o,
+                        float *state_out, void *cuda_stream) {
+  if (T < 0) return GDN_ERR_INVALID_ARG;
+  const long long rows = cu_seqlens ? (long long)T : (long long)n_seq * T;
+  gdn_status s = check_common(q, k, v, g, beta, o, n_seq, H, d_k, d_v, dt, gk, qdq, rows);
+  if (s != GDN_OK) return s;
+  int kind = 0, group = 32;
+  if (!qdq_params(qdq, d_v, &kind, &group)) return GDN_ERR_UNSUPPORTED;
+  if (n_seq == 0) return GDN_OK;
+  if (!state_out || !aligned(state_out, 16)) return GDN_ERR_INVALID_ARG;
+  if (state_in && !aligned(state_in, 16)) return GDN_ERR_INVALID_ARG;
+  if (cu_seqlens && !aligned(cu_seqlens, 4)) return GDN_ERR_INVALID_ARG;
+  // Total token rows must index within 64-bit element offsets comfortably.
+  if (rows * H * 128 > (1LL << 46)) return GDN_ERR_UNSUPPORTED;
+  unsigned *err = nullptr;
+  if ((s = err_word(&err)) != GDN_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  const bool pk = gk == GDN_GATE_PER_KEY;
+  // Kernel choice by specialisation (tc_path); the Neumann solve runs on the
+  // CUDA-core kernel for every dtype.  Both compute the same chunked algebra.
+  if (neu_m == 0 && tc_path(dt, gk, d_k, d_v))
+    return launch_prefill_tc(q, k, v, g, beta, state_in, cu_seqlens, n_seq, T, H, kind, group, o,
+                             state_out, err, st);
+  if (dt == GDN_DTYPE_BF16)
+    return launch_prefill_simt<__nv_bfloat16>(q, k, v, g, beta, state_in, cu_seqlens, n_seq, T,
+                                              H, d_k, d_v, pk, kind, group, o, state_out, err,
+                                              neu_m, st);
+  return launch_prefill_simt<float>(q, k, v, g, beta, state_in, cu_seqlens, n_seq, T, H, d_k,
+                                    d_v, pk, kind, group, o, state_out, err, neu_m, st);
+}
+
 }  // namespace
 
 extern "C" {
@@ -433,34 +485,20 @@ gdn_status gdn_prefill(const void *q, const void *k, const void *v, const float 
                        int n_seq, int T, int H, int d_k, int d_v, gdn_dtype dt,
                        gdn_gate_kind gk, gdn_qdq_mode qdq, void *o, float *state_out,
                        void *cuda_stream) {
-  if (T < 0) return GDN_ERR_INVALID_ARG;
-  const long long rows = cu_seqlens ? (long long)T : (long long)n_seq * T;
-  gdn_status s = check_common(q, k, v, g, beta, o, n_seq, H, d_k, d_v, dt, gk, qdq, rows);
-  if (s != GDN_OK) return s;
-  int kind = 0, group = 32;
-  if (!qdq_params(qdq, d_v, &kind, &group)) return GDN_ERR_UNSUPPORTED;
-  if (n_seq == 0) return GDN_OK;
-  if (!state_out || !aligned(state_out, 16)) return GDN_ERR_INVALID_ARG;
-  if (state_in && !aligned(state_in, 16)) return GDN_ERR_INVALID_ARG;
-  if (cu_seqlens && !aligned(cu_seqlens, 4)) return GDN_ERR_INVALID_ARG;
-  // Total token rows must index within 64-bit element offsets comfortably.
-  if (rows * H * 128 > (1LL << 46)) return GDN_ERR_UNSUPPORTED;
-  unsigned *err = nullptr;
-  if ((s = err_word(&err)) != GDN_OK) return s;
-  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
-  const bool pk = gk == GDN_GATE_PER_KEY;
-  // Kernel choice by specialisation: bf16 GDN at d_k = d_v = 128 runs on the
-  // tensor cores; fp32 inputs (whose 1e-5 tolerance the fp16 operand splits
-  // cannot promise), per-key (KDA) gates and d = 64 run on the CUDA-core
-  // kernel.  Both compute the same chunked algebra.
-  if (tc_path(dt, gk, d_k, d_v))
-    return launch_prefill_tc(q, k, v, g, beta, state_in, cu_seqlens, n_seq, T, H, kind, group, o,
-                             state_out, err, st);
-  if (dt == GDN_DTYPE_BF16)
-    return launch_prefill_simt<__nv_bfloat16>(q, k, v, g, beta, state_in, cu_seqlens, n_seq, T,
-                                              H, d_k, d_v, pk, kind, group, o, state_out, err, st);
-  return launch_prefill_simt<float>(q, k, v, g, beta, state_in, cu_seqlens, n_seq, T, H, d_k,
-                                    d_v, pk, kind, group, o, state_out, err, st);
+  return prefill_impl(q, k, v, g, beta, state_in, cu_seqlens, n_seq, T, H, d_k, d_v, dt, gk, qdq,
+                      0, o, state_out, cuda_stream);
+}
+
+gdn_status gdn_prefill_neumann(const void *q, const void *k, const void *v, const float *g,
+                               const float *beta, const float *state_in,
+                               const int32_t *cu_seqlens, int n_seq, int T, int H, int d_k,
+                               int d_v, gdn_dtype dt, gdn_gate_kind gk, gdn_qdq_mode qdq,
+                               int degree, void *o, float *state_out, void *cuda_stream) {
+  int m = 0;
+  while (m < 6 && degree != (1 << (m + 1)) - 1) ++m;
+  if (m == 6) return GDN_ERR_INVALID_ARG;  // degree not in {1, 3, 7, 15, 31, 63}
+  return prefill_impl(q, k, v, g, beta, state_in, cu_seqlens, n_seq, T, H, d_k, d_v, dt, gk, qdq,
+                      m + 1, o, state_out, cuda_stream);
 }
 
 int gdn_prefill_schedule(int n_seq, int H, int d_k, int d_v, gdn_dtype dt, gdn_gate_kind gk) {

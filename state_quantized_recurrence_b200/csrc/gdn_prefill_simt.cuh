@@ -30,7 +30,9 @@ constexpr int kThreads = 256;
 constexpr int LDV = 68;  // row stride (floats) of [64 x 64] tiles
 constexpr int LDA = 66;  // row stride of A / Aqk
 
-template <int DK>
+constexpr int LDT = 68;  // row stride of the Neumann product-form matrices
+
+template <int DK, bool NEU = false>
 struct Smem {
   static constexpr int LDK = DK + 4;
   static constexpr int kRegion = (64 * LDK > 2 * 64 * LDA) ? 64 * LDK : 2 * 64 * LDA;
@@ -48,15 +50,53 @@ struct Smem {
   static constexpr int oGref = oEnr + DK;
   static constexpr int oGn = oGref + DK;
   static constexpr int oRed = oGn + DK;
-  static constexpr int kFloats = oRed + 32;
+  // Neumann solve only: T and the running power X^(2^i), [64 x LDT] each
+  static constexpr int oT = (oRed + 32 + 3) & ~3;
+  static constexpr int oP = oT + 64 * LDT;
+  static constexpr int kFloats = NEU ? oP + 64 * LDT : oRed + 32;
   static constexpr size_t kBytes = sizeof(float) * kFloats;
 };
+
+static_assert(Smem<128, true>::kBytes <= 232448, "Neumann variant exceeds shared memory");
+static_assert(Smem<128, true>::oT % 4 == 0 && (LDT * 4) % 16 == 0, "float4 rows of T and P");
 
 __device__ __forceinline__ float dot4(float4 a, float4 b) {
   return a.x * b.x + a.y * b.y + a.z * b.z + a.w * b.w;
 }
 
-template <typename Tin, int DK, bool PER_KEY>
+// C = M1 M2 for lower-triangular 64 x 64 operands (row stride LDT), the 4 x 4
+// block (rows 4 R .., columns 4 C ..) of this thread into `acc` (zero above
+// the diagonal): terms with i outside [4 C, 4 R + 3] vanish because the
+// operands' upper triangles are zero.
+__device__ __forceinline__ void lower_mul_block(const float *M1, const float *M2, int R, int C,
+                                                float (&acc)[4][4]) {
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) acc[a][b] = 0.0f;
+  if (C > R) return;
+  for (int i0 = 4 * C; i0 <= 4 * R; i0 += 4) {
+    float4 m2[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) m2[e] = *reinterpret_cast<const float4 *>(M2 + (i0 + e) * LDT + 4 * C);
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      const float4 m1 = *reinterpret_cast<const float4 *>(M1 + (4 * R + a) * LDT + i0);
+      const float w[4] = {m1.x, m1.y, m1.z, m1.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        acc[a][0] += w[e] * m2[e].x; acc[a][1] += w[e] * m2[e].y;
+        acc[a][2] += w[e] * m2[e].z; acc[a][3] += w[e] * m2[e].w;
+      }
+    }
+  }
+}
+
+// NEU: the approximate solve of the GDN/KDA approximate-inverse PR (#2507,
+// What section: an explicit Neumann polynomial degree) in place of the exact
+// one: T = sum_{n <= d} (-A)^n with d = 2^neu_m - 1, evaluated as
+// prod_{i < neu_m} (I + X^(2^i)), X = -A.
+template <typename Tin, int DK, bool PER_KEY, bool NEU>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
                     const Tin *__restrict__ v, const float *__restrict__ g,
@@ -65,8 +105,8 @@ prefill_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
                     const int *__restrict__ cu_seqlens, int T, int H, int DV,
                     float scale, int qdq_kind, int qdq_group,
                     Tin *__restrict__ o, float *__restrict__ state_out,
-                    unsigned *__restrict__ err) {
-  using L = Smem<DK>;
+                    unsigned *__restrict__ err, int neu_m) {
+  using L = Smem<DK, NEU>;
   constexpr int LDK = L::LDK;
   extern __shared__ __align__(16) float sm[];
   float *sK = sm + L::oK, *sX = sm + L::oX, *sQ = sm + L::oQ, *sR = sm + L::oR;
@@ -264,29 +304,90 @@ prefill_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
     }
     __syncthreads();
 
-    // ---- P5: [W | U] = (I + A)^-1 RHS by forward substitution, one column
-    //      per thread held in registers ----
-    if (tid < DK + 64) {
-      float *colp = tid < DK ? sK + tid : sV + (tid - DK);
-      const int ld = tid < DK ? LDK : LDV;
-      float x[kChunk];
+    if (NEU) {
+      // ---- P5 (Neumann): T = prod_{i < m} (I + X^(2^i)), X = -A, then
+      //      [W | U] = T RHS, one column per thread held in registers ----
+      float *sT = sm + L::oT, *sP = sm + L::oP;
+      for (int idx = tid; idx < 64 * 64; idx += kThreads) {
+        const int r = idx >> 6, c = idx & 63;
+        const float x = c < r ? -sA[r * LDA + c] : 0.0f;
+        sP[r * LDT + c] = x;
+        sT[r * LDT + c] = r == c ? 1.0f : x;
+      }
+      const int R = tid >> 4, C = tid & 15;
+      for (int i = 1; i < neu_m; ++i) {
+        float acc[4][4];
+        __syncthreads();
+        lower_mul_block(sP, sP, R, C, acc);  // P <- P P
+        __syncthreads();
+        if (C <= R) {
 #pragma unroll
-      for (int r = 0; r < kChunk; ++r) {
-        if (r < n) {
-          float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
-          const float *arow = sA + r * LDA;
+          for (int a = 0; a < 4; ++a)
+            *reinterpret_cast<float4 *>(sP + (4 * R + a) * LDT + 4 * C) =
+                make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
+        }
+        __syncthreads();
+        lower_mul_block(sT, sP, R, C, acc);  // T <- T + T P
+        __syncthreads();
+        if (C <= R) {
 #pragma unroll
-          for (int i = 0; i + 1 < r; i += 2) {
-            float2 aa = *reinterpret_cast<const float2 *>(arow + i);
-            if (i & 2) { p2 += aa.x * x[i]; p3 += aa.y * x[i + 1]; }
-            else       { p0 += aa.x * x[i]; p1 += aa.y * x[i + 1]; }
+          for (int a = 0; a < 4; ++a) {
+            float4 *t = reinterpret_cast<float4 *>(sT + (4 * R + a) * LDT + 4 * C);
+            const float4 tv = *t;
+            *t = make_float4(tv.x + acc[a][0], tv.y + acc[a][1], tv.z + acc[a][2], tv.w + acc[a][3]);
           }
-          if (r & 1) p0 += arow[r - 1] * x[r - 1];
-          const float xr = colp[r * ld] - ((p0 + p1) + (p2 + p3));
-          x[r] = xr;
-          colp[r * ld] = xr;
-        } else {
-          x[r] = 0.0f;
+        }
+      }
+      __syncthreads();
+      if (tid < DK + 64) {
+        float *colp = tid < DK ? sK + tid : sV + (tid - DK);
+        const int ld = tid < DK ? LDK : LDV;
+        float x[kChunk];
+#pragma unroll
+        for (int r = 0; r < kChunk; ++r) x[r] = colp[r * ld];
+        // rows past n: T is the identity there and the right-hand side zero
+#pragma unroll
+        for (int r = 0; r < kChunk; ++r) {
+          const float *trow = sT + r * LDT;
+          float p0 = 0.f, p1 = 0.f;
+#pragma unroll
+          for (int i = 0; i <= r; i += 2) {
+            if (i + 1 <= r) {
+              const float2 tt = *reinterpret_cast<const float2 *>(trow + i);
+              p0 += tt.x * x[i];
+              p1 += tt.y * x[i + 1];
+            } else {
+              p0 += trow[i] * x[i];
+            }
+          }
+          colp[r * ld] = p0 + p1;
+        }
+      }
+    } else {
+      // ---- P5: [W | U] = (I + A)^-1 RHS by forward substitution, one column
+      //      per thread held in registers ----
+      if (tid < DK + 64) {
+        float *colp = tid < DK ? sK + tid : sV + (tid - DK);
+        const int ld = tid < DK ? LDK : LDV;
+        float x[kChunk];
+#pragma unroll
+        for (int r = 0; r < kChunk; ++r) {
+          if (r < n) {
+            float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
+            const float *arow = sA + r * LDA;
+#pragma unroll
+            for (int i = 0; i + 1 < r; i += 2) {
+              float2 aa = *reinterpret_cast<const float2 *>(arow + i);
+              if (i & 2) { p2 += aa.x * x[i]; p3 += aa.y * x[i + 1]; }
+              else       { p0 += aa.x * x[i]; p1 += aa.y * x[i + 1]; }
+            }
+            if (r & 1) p0 += arow[r - 1] * x[r - 1];
+            const float xr = colp[r * ld] - ((p0 + p1) + (p2 + p3));
+            x[r] = xr;
+            colp[r * ld] = xr;
+          } else {
+            x[r] = 0.0f;
+          }
         }
       }
     }

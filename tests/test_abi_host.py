@@ -36,6 +36,8 @@ def lib():
     P, I = ctypes.c_void_p, ctypes.c_int
     L.gdn_prefill.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P, P, P]
     L.gdn_prefill.restype = I
+    L.gdn_prefill_neumann.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, P, P, P]
+    L.gdn_prefill_neumann.restype = I
     L.gdn_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, P, P]
     L.gdn_decode.restype = I
     L.gdn_decode_packed.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, P]
@@ -87,6 +89,16 @@ def pf(lib, **kw):
                            a["qdq"], a["o"], a["state_out"], a["stream"])
 
 
+def pn(lib, degree=3, **kw):
+    a = dict(q=A, k=A, v=A, g=A, beta=A, state_in=None, cu=None, n_seq=2, T=64, H=4, d_k=128,
+             d_v=128, dt=BF16, gk=0, qdq=1, o=A, state_out=A, stream=None)
+    a.update(kw)
+    return lib.gdn_prefill_neumann(a["q"], a["k"], a["v"], a["g"], a["beta"], a["state_in"],
+                                   a["cu"], a["n_seq"], a["T"], a["H"], a["d_k"], a["d_v"],
+                                   a["dt"], a["gk"], a["qdq"], degree, a["o"], a["state_out"],
+                                   a["stream"])
+
+
 def dc(lib, **kw):
     a = dict(q=A, k=A, v=A, g=A, beta=A, state=A, n_seq=2, H=4, d_k=128, d_v=128, dt=BF16, gk=0,
              qdq=2, o=A, stream=None)
@@ -115,7 +127,7 @@ def cv(lib, unpack=False, **kw):
                               a["d_v"], a["qdq"], a["stream"])
 
 
-@pytest.mark.parametrize("call", [pf, dc, dp])
+@pytest.mark.parametrize("call", [pf, pn, dc, dp])
 def test_validation_errors(lib, call):
     assert call(lib, n_seq=-1) == INVALID
     assert call(lib, H=0) == INVALID
@@ -139,6 +151,14 @@ def test_prefill_specific_errors(lib):
     assert pf(lib, state_out=A + 4) == INVALID
     assert pf(lib, state_in=A + 4) == INVALID
     assert pf(lib, cu=A + 2) == INVALID
+
+
+@pytest.mark.parametrize("degree", [-1, 0, 2, 4, 5, 30, 64, 127])
+def test_neumann_degree_rejected(lib, degree):
+    """Only 2^m - 1 for m = 1..6: any other degree is refused before a
+    launch, never rounded to a supported one."""
+    assert pn(lib, degree=degree) == INVALID
+    assert pn(lib, degree=degree, n_seq=0) == INVALID
 
 
 def test_decode_specific_errors(lib):
