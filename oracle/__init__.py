@@ -4,13 +4,16 @@ TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and
 the benchmark's CPU-baseline leg may import this package; the product path
 (``state_quantized_recurrence_b200``) never does, and the two share no code.
 
-Two modes:
+Modes:
 
 * :func:`recurrence` - the definition: the fp64 token-by-token gated delta
   rule with the fp32 QDQ codecs at chunk boundaries / after decode tokens,
   in plain C (``gdn_oracle.c``), OpenMP over independent (sequence, head).
 * :func:`oracle.chunked.chunked_wy` - the 64-token chunked WY form in fp64
-  numpy, used to pin the chunked algebra against the token recurrence.
+  numpy, used to pin the chunked algebra against the token recurrence (and,
+  with ``solve=("neumann", d)``, the approximate solve).
+* :func:`oracle.backward.backward` - the fp64 reverse pass of the token
+  recurrence with the state QDQ passed straight through.
 
 Pins: every function here is checked by ``tests/test_oracle_*.py`` against
 closed forms, invariants, special cases and library routines (see the
