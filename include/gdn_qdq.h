@@ -49,6 +49,7 @@
 #ifndef GDN_QDQ_H_
 #define GDN_QDQ_H_
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -197,6 +198,40 @@ gdn_status gdn_prefill_neumann(const void *q, const void *k, const void *v,
                                gdn_dtype dt, gdn_gate_kind gk, gdn_qdq_mode qdq,
                                int degree, void *o, float *state_out,
                                void *cuda_stream);
+
+/*
+ * gdn_prefill_backward - gradients of one gdn_prefill call (the same
+ * inputs, layout and qdq mode) for training with the state QAT of the
+ * pages (PR #2497, What section: fake quantization of the recurrent state;
+ * the QDQ is passed straight through in the backward pass, STE).
+ *
+ * d_o: upstream gradient of o, dtype dt, shaped like o.  dstate_out: fp32
+ *   gradient of state_out [n_seq, H, d_k, d_v], or NULL for zero.
+ * Outputs (fp32, caller-owned device memory, shaped like the matching input):
+ *   dq, dk [.., H, d_k]; dv [.., H, d_v]; dg [.., H] or [.., H, d_k]; dbeta
+ *   [.., H]; dstate_in [n_seq, H, d_k, d_v] (the gradient of state_in; of
+ *   the zero state when state_in is NULL).  dq, dk, dg and dbeta are zeroed
+ *   on the stream and accumulated.
+ * workspace: caller-owned device memory of at least
+ *   gdn_prefill_backward_workspace_bytes(n_seq, T, H, d_k, d_v,
+ *   cu_seqlens != NULL) bytes, 16-byte aligned; its contents are scratch.
+ *   The forward recurrence is recomputed from state_in (in fp32, with the
+ *   QDQ at every chunk end), so no forward activations are needed.
+ * Errors: as gdn_prefill; a missing, misaligned or short workspace, or a
+ *   missing output, is GDN_ERR_INVALID_ARG.  Runs on the CUDA cores for
+ *   every dtype, gate kind and shape.
+ */
+size_t gdn_prefill_backward_workspace_bytes(int n_seq, int T, int H, int d_k,
+                                            int d_v, int packed);
+gdn_status gdn_prefill_backward(const void *q, const void *k, const void *v,
+                                const float *g, const float *beta,
+                                const float *state_in, const int32_t *cu_seqlens,
+                                int n_seq, int T, int H, int d_k, int d_v,
+                                gdn_dtype dt, gdn_gate_kind gk, gdn_qdq_mode qdq,
+                                const void *d_o, const float *dstate_out,
+                                void *workspace, size_t workspace_bytes,
+                                float *dq, float *dk, float *dv, float *dg,
+                                float *dbeta, float *dstate_in, void *cuda_stream);
 
 /*
  * gdn_prefill_schedule - which prefill kernel gdn_prefill launches for these

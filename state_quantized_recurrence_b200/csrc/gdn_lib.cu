@@ -11,6 +11,7 @@
 
 #include "gdn_qdq.h"
 #include "gdn_common.cuh"
+#include "gdn_backward.cuh"
 #include "gdn_decode.cuh"
 #include "gdn_prefill_simt.cuh"
 #include "gdn_prefill_pair.cuh"
@@ -362,6 +363,53 @@ gdn_status launch_prefill_tc(const void *q, const void *k, const void *v, const 
 #undef GDN_TC
 }
 
+// ---- backward (CUDA cores) ------------------------------------------------
+// Workspace: every chunk's starting state per (slot, head, value tile), plus
+// one chunk of per-token states per CTA.  Packed sequences take chunk slots
+// s + cu[s] / 64 onwards, at most n_seq + T / 64 in all.
+long long backward_ws_floats(int n_seq, long long T, int H, int d_k, int d_v, bool packed,
+                             long long *chunk_floats) {
+  const long long nvt = d_v / 64, tile = (long long)d_k * 64;
+  const long long slots = packed ? n_seq + T / 64 : (long long)n_seq * ((T + 63) / 64);
+  const long long ctas = (long long)n_seq * H * nvt;
+  *chunk_floats = slots * H * nvt * tile;
+  return *chunk_floats + ctas * 64 * tile;
+}
+
+template <typename Tin, int DK, bool PK, int QK, int GR>
+gdn_status launch_bwd_one(const void *q, const void *k, const void *v, const float *g,
+                          const float *beta, const float *state_in, const int32_t *cu, int T,
+                          int H, int d_v, const void *d_o, const float *dstate_out, float *ws,
+                          long long chunk_floats, float *dq, float *dk, float *dv, float *dg,
+                          float *dbeta, float *dstate_in, unsigned *err, unsigned blocks,
+                          cudaStream_t st) {
+  const float scale = (float)(1.0 / sqrt((double)DK));
+  gdn::bwd::prefill_backward_kernel<Tin, DK, PK, QK, GR><<<blocks, gdn::bwd::kThreads, 0, st>>>(
+      static_cast<const Tin *>(q), static_cast<const Tin *>(k), static_cast<const Tin *>(v), g,
+      beta, state_in, cu, T, H, d_v, scale, static_cast<const Tin *>(d_o), dstate_out, ws,
+      ws + chunk_floats, dq, dk, dv, dg, dbeta, dstate_in, err);
+  return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+template <typename Tin, int DK, bool PK>
+gdn_status launch_bwd_qdq(int kind, int group, const void *q, const void *k, const void *v,
+                          const float *g, const float *beta, const float *state_in,
+                          const int32_t *cu, int T, int H, int d_v, const void *d_o,
+                          const float *dstate_out, float *ws, long long chunk_floats, float *dq,
+                          float *dk, float *dv, float *dg, float *dbeta, float *dstate_in,
+                          unsigned *err, unsigned blocks, cudaStream_t st) {
+#define GDN_BW(QK, GR)                                                                            \
+  launch_bwd_one<Tin, DK, PK, QK, GR>(q, k, v, g, beta, state_in, cu, T, H, d_v, d_o, dstate_out, \
+                                      ws, chunk_floats, dq, dk, dv, dg, dbeta, dstate_in, err,     \
+                                      blocks, st)
+  if (kind == gdn::kQdqNone) return GDN_BW(gdn::kQdqNone, 32);
+  if (kind == gdn::kQdqFp8Tile) return GDN_BW(gdn::kQdqFp8Tile, 32);
+  if (group == 16) return GDN_BW(gdn::kQdqInt8, 16);
+  if (group == 64) return GDN_BW(gdn::kQdqInt8, 64);
+  return GDN_BW(gdn::kQdqInt8, 32);
+#undef GDN_BW
+}
+
 // Validation and kernel choice shared by gdn_prefill and gdn_prefill_neumann
 // (neu_m = 0: exact solve; >= 1: Neumann degree 2^neu_m - 1).
 gdn_status prefill_impl(const void *q, const void *k, const void *v, const float *g,
@@ -499,6 +547,73 @@ gdn_status gdn_prefill_neumann(const void *q, const void *k, const void *v, cons
   if (m == 6) return GDN_ERR_INVALID_ARG;  // degree not in {1, 3, 7, 15, 31, 63}
   return prefill_impl(q, k, v, g, beta, state_in, cu_seqlens, n_seq, T, H, d_k, d_v, dt, gk, qdq,
                       m + 1, o, state_out, cuda_stream);
+}
+
+size_t gdn_prefill_backward_workspace_bytes(int n_seq, int T, int H, int d_k, int d_v,
+                                            int packed) {
+  if (n_seq < 0 || T < 0 || H <= 0) return 0;
+  if ((d_k != 64 && d_k != 128) || (d_v != 64 && d_v != 128)) return 0;
+  long long chunk_floats = 0;
+  return (size_t)backward_ws_floats(n_seq, T, H, d_k, d_v, packed != 0, &chunk_floats) *
+         sizeof(float);
+}
+
+gdn_status gdn_prefill_backward(const void *q, const void *k, const void *v, const float *g,
+                                const float *beta, const float *state_in,
+                                const int32_t *cu_seqlens, int n_seq, int T, int H, int d_k,
+                                int d_v, gdn_dtype dt, gdn_gate_kind gk, gdn_qdq_mode qdq,
+                                const void *d_o, const float *dstate_out, void *workspace,
+                                size_t workspace_bytes, float *dq, float *dk, float *dv,
+                                float *dg, float *dbeta, float *dstate_in, void *cuda_stream) {
+  if (T < 0) return GDN_ERR_INVALID_ARG;
+  const long long rows = cu_seqlens ? (long long)T : (long long)n_seq * T;
+  gdn_status s = check_common(q, k, v, g, beta, d_o, n_seq, H, d_k, d_v, dt, gk, qdq, rows);
+  if (s != GDN_OK) return s;
+  int kind = 0, group = 32;
+  if (!qdq_params(qdq, d_v, &kind, &group)) return GDN_ERR_UNSUPPORTED;
+  if (n_seq == 0) return GDN_OK;
+  if (!dstate_in || !aligned(dstate_in, 16)) return GDN_ERR_INVALID_ARG;
+  if (state_in && !aligned(state_in, 16)) return GDN_ERR_INVALID_ARG;
+  if (dstate_out && !aligned(dstate_out, 16)) return GDN_ERR_INVALID_ARG;
+  if (cu_seqlens && !aligned(cu_seqlens, 4)) return GDN_ERR_INVALID_ARG;
+  if (rows > 0 && (!dq || !dk || !dv || !dg || !dbeta)) return GDN_ERR_INVALID_ARG;
+  if (!aligned(dq, 4) || !aligned(dk, 4) || !aligned(dv, 16) || !aligned(dg, 4) ||
+      !aligned(dbeta, 4))
+    return GDN_ERR_INVALID_ARG;
+  if (rows * H * 128 > (1LL << 46)) return GDN_ERR_UNSUPPORTED;
+  long long chunk_floats = 0;
+  const long long need = backward_ws_floats(n_seq, T, H, d_k, d_v, cu_seqlens != nullptr,
+                                            &chunk_floats);
+  if (!workspace || !aligned(workspace, 16) || workspace_bytes < (size_t)need * sizeof(float))
+    return GDN_ERR_INVALID_ARG;
+  const long long blocks = (long long)n_seq * H * (d_v / 64);
+  if (blocks > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+  unsigned *err = nullptr;
+  if ((s = err_word(&err)) != GDN_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  const bool pk = gk == GDN_GATE_PER_KEY;
+  // sums over value tiles are accumulated with atomic adds
+  if (rows > 0) {
+    const size_t kb = (size_t)rows * H * d_k * sizeof(float);
+    if (cudaMemsetAsync(dq, 0, kb, st) != cudaSuccess ||
+        cudaMemsetAsync(dk, 0, kb, st) != cudaSuccess ||
+        cudaMemsetAsync(dg, 0, pk ? kb : (size_t)rows * H * sizeof(float), st) != cudaSuccess ||
+        cudaMemsetAsync(dbeta, 0, (size_t)rows * H * sizeof(float), st) != cudaSuccess)
+      return GDN_ERR_CUDA;
+  }
+  float *ws = static_cast<float *>(workspace);
+  const unsigned nb = (unsigned)blocks;
+#define GDN_BQ(TIN, DK, PK)                                                                       \
+  launch_bwd_qdq<TIN, DK, PK>(kind, group, q, k, v, g, beta, state_in, cu_seqlens, T, H, d_v, d_o, \
+                              dstate_out, ws, chunk_floats, dq, dk, dv, dg, dbeta, dstate_in, err, \
+                              nb, st)
+  if (dt == GDN_DTYPE_BF16) {
+    if (d_k == 128) return pk ? GDN_BQ(__nv_bfloat16, 128, true) : GDN_BQ(__nv_bfloat16, 128, false);
+    return pk ? GDN_BQ(__nv_bfloat16, 64, true) : GDN_BQ(__nv_bfloat16, 64, false);
+  }
+  if (d_k == 128) return pk ? GDN_BQ(float, 128, true) : GDN_BQ(float, 128, false);
+  return pk ? GDN_BQ(float, 64, true) : GDN_BQ(float, 64, false);
+#undef GDN_BQ
 }
 
 int gdn_prefill_schedule(int n_seq, int H, int d_k, int d_v, gdn_dtype dt, gdn_gate_kind gk) {

@@ -161,6 +161,50 @@ def test_neumann_degree_rejected(lib, degree):
     assert pn(lib, degree=degree, n_seq=0) == INVALID
 
 
+def bw(lib, ws_bytes=None, **kw):
+    import ctypes as C
+    lib.gdn_prefill_backward_workspace_bytes.argtypes = [C.c_int] * 6
+    lib.gdn_prefill_backward_workspace_bytes.restype = C.c_size_t
+    P, I = C.c_void_p, C.c_int
+    lib.gdn_prefill_backward.argtypes = [P] * 7 + [I] * 8 + [P, P, P, C.c_size_t] + [P] * 7
+    lib.gdn_prefill_backward.restype = I
+    a = dict(q=A, k=A, v=A, g=A, beta=A, state_in=None, cu=None, n_seq=2, T=64, H=4, d_k=128,
+             d_v=128, dt=BF16, gk=0, qdq=1, d_o=A, dso=None, ws=A, dq=A, dk=A, dv=A, dg=A,
+             dbeta=A, dsi=A, stream=None)
+    a.update(kw)
+    need = lib.gdn_prefill_backward_workspace_bytes(a["n_seq"], a["T"], a["H"], a["d_k"],
+                                                    a["d_v"], int(a["cu"] is not None))
+    return lib.gdn_prefill_backward(
+        a["q"], a["k"], a["v"], a["g"], a["beta"], a["state_in"], a["cu"], a["n_seq"], a["T"],
+        a["H"], a["d_k"], a["d_v"], a["dt"], a["gk"], a["qdq"], a["d_o"], a["dso"], a["ws"],
+        need if ws_bytes is None else ws_bytes, a["dq"], a["dk"], a["dv"], a["dg"], a["dbeta"],
+        a["dsi"], a["stream"])
+
+
+def test_backward_workspace_and_errors(lib):
+    """Workspace size formula (chunk-start states per slot and value tile,
+    plus one chunk of token states per CTA) and the checks made before any
+    launch."""
+    lib.gdn_prefill_backward_workspace_bytes.argtypes = [ctypes.c_int] * 6
+    lib.gdn_prefill_backward_workspace_bytes.restype = ctypes.c_size_t
+    tile = 128 * 64 * 4
+    # dense: 2 sequences x ceil(100 / 64) = 4 slots, 4 heads, 2 tiles; 16 CTAs
+    assert lib.gdn_prefill_backward_workspace_bytes(2, 100, 4, 128, 128, 0) == \
+        tile * (4 * 4 * 2 + 16 * 64)
+    # packed: n_seq + T / 64 slots
+    assert lib.gdn_prefill_backward_workspace_bytes(3, 200, 1, 128, 64, 1) == \
+        tile * ((3 + 3) * 1 * 1 + 3 * 64)
+    assert lib.gdn_prefill_backward_workspace_bytes(2, 64, 4, 96, 128, 0) == 0
+    assert bw(lib, ws_bytes=1) == INVALID            # workspace too small
+    assert bw(lib, ws=None) == INVALID
+    assert bw(lib, ws=A + 4) == INVALID              # 16-byte alignment
+    assert bw(lib, dsi=None) == INVALID
+    assert bw(lib, dq=None) == INVALID
+    assert bw(lib, d_o=None) == INVALID
+    assert bw(lib, d_k=96) == UNSUPPORTED
+    assert bw(lib, n_seq=0) == OK
+
+
 def test_decode_specific_errors(lib):
     assert dc(lib, state=None) == INVALID
     assert dc(lib, state=A + 4) == INVALID
