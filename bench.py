@@ -90,6 +90,19 @@ def prefill_bytes(tokens, n_states, H, dk, dv, in_bytes, state_in: bool, per_key
     return b
 
 
+def backward_bytes(tokens, n_states, H, dk, dv, in_bytes, state_in: bool, per_key: bool) -> int:
+    """Algorithmic HBM bytes of one gdn_prefill_backward call: q, k, v and
+    d_o read (in dtype), g and beta read, the initial state read; dq, dk, dv,
+    dg, dbeta and dstate_in written in fp32 (the recomputation's re-reads and
+    the workspace traffic are not algorithmic)."""
+    tok = tokens * H
+    g_el = dk if per_key else 1
+    b = tok * (2 * dk + 2 * dv) * in_bytes + tok * 4 * (g_el + 1)
+    b += tok * 4 * (2 * dk + dv + g_el + 1)
+    b += n_states * H * dk * dv * 4 * (2 if state_in else 1)
+    return b
+
+
 def prefill_flops(tokens, H, dk, dv, C=64) -> int:
     """Dense algorithmic flops of the chunked WY form: per chunk of C tokens
     K K^T, Q K^T and W = T (bK): 3 * 2*C*C*d_k; U = T (bV) and Aqk Vn:
@@ -249,6 +262,87 @@ def cpu_baseline_decode(case, inp, state) -> dict:
             "seconds": round(dt, 3)}
 
 
+def cpu_baseline_backward(case, inp, d_o, max_tokens: int = 512) -> dict:
+    """The backward oracle (fp64 numpy, one (sequence, head) at a time) on
+    the first `max_tokens` tokens of the first sequence, all heads."""
+    from oracle import backward as obw
+    n = min(max_tokens, int(inp["lengths"][0]))
+    sl = (slice(0, 1), slice(0, n))
+    st_in = inp["state_in"][0:1] if inp["state_in"] is not None else None
+    t0 = time.perf_counter()
+    obw.backward(inp["q"][sl], inp["k"][sl], inp["v"][sl], inp["g"][sl], inp["beta"][sl], st_in,
+                 [0, n], d_o[sl], None, per_key_gate=case.gate == "per_key", qdq=case.qdq)
+    dt = time.perf_counter() - t0
+    return {"value": n / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} tokens of 1 of {case.n_seq} sequences x {case.H} heads, fp64 token "
+                      f"reverse pass (numpy, one thread), {case.qdq} straight through",
+            "seconds": round(dt, 3)}
+
+
+def measure_backward(args, dist, dev, stream, sampler, peaks, case, steps, warmup) -> dict:
+    """Time `steps` gdn_prefill_backward calls of `case` (inputs, upstream
+    gradient and workspace resident in HBM)."""
+    import torch
+
+    import gdn_synth as gs
+    import state_quantized_recurrence_b200 as sqr
+
+    inp = gs.generate(case)
+    gen = torch.Generator().manual_seed(case.seed + 500)
+    d_o = torch.randn(inp["v"].shape, generator=gen).to(inp["q"].dtype)
+    d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    d_o_dev = d_o.to(dev)
+    T_arg = int(sum(inp["lengths"])) if d["cu_seqlens"] is not None else case.T
+    need = int(sqr.lib.gdn_prefill_backward_workspace_bytes(
+        case.n_seq, T_arg, case.H, case.d_k, case.d_v, int(d["cu_seqlens"] is not None)))
+    ws = torch.empty(need, dtype=torch.uint8, device=dev)
+
+    def step():
+        return sqr.gdn_prefill_backward(d["q"], d["k"], d["v"], d["g"], d["beta"], d_o_dev,
+                                        d["state_in"], d["cu_seqlens"], None, qdq=case.qdq,
+                                        workspace=ws)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    sqr.check_last_error(where=f"{case.name} backward warm-up")
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    t_wall0 = time.time()
+    ev0.record(stream)
+    for _ in range(steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    t_wall1 = time.time()
+    dist.barrier()
+    ms = dist.max(ev0.elapsed_time(ev1) / steps)
+    tokens = int(sum(inp["lengths"]))
+    nbytes = backward_bytes(tokens, case.n_seq, case.H, case.d_k, case.d_v,
+                            2 if case.dtype == "bf16" else 4, inp["state_in"] is not None,
+                            case.gate == "per_key")
+    gbs = nbytes / (ms / 1e3) / 1e9
+    res = {
+        "metric": "prefill backward tokens/s (straight-through state QDQ)",
+        "workload": f"{case.name}: n_seq={case.n_seq} H={case.H} tokens={tokens} d={case.d_k}, "
+                    f"{case.dtype}, {case.gate} gate, {case.qdq}, random d_o, no dstate_out",
+        "value": round(dist.world * tokens / (ms / 1e3), 1), "unit": "tokens/s",
+        "ms_per_step": round(ms, 4), "steps": steps,
+        "kernel": "bwd::prefill_backward_kernel (FFMA, token-reverse with chunk checkpoints)",
+        "workspace_bytes": need,
+        "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 5), "traffic": None,
+                     "bytes_per_launch": nbytes, "peak_source": peaks["source"]},
+        "gpu_launches": steps, "clocks": sampler.summary(t_wall0, t_wall1),
+    }
+    if dist.rank == 0 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline_backward(case, inp, d_o)
+    del d, d_o_dev, ws
+    torch.cuda.empty_cache()
+    return res
+
+
 def measure_prefill(args, dist, dev, stream, sampler, peaks, case, steps, warmup,
                     traffic_key=None, keep=False, cpu=False):
     """Time `steps` gdn_prefill calls of `case` (inputs resident in HBM).
@@ -379,6 +473,12 @@ def run_ours(args, dist: Dist) -> dict:
             others[name] = measure_prefill(args, dist, dev, stream, sampler, peaks, c,
                                            max(3, min(args.steps, 10)), args.warmup, cpu=True)
 
+    # ---------------- backward (straight-through QDQ) on the prefill workload ----------------
+    bwd = None
+    if not args.only and not args.small and not args.no_others:
+        bwd = measure_backward(args, dist, dev, stream, sampler, peaks, gs.CONFIGS["gdn_prefill"],
+                               3, 3)
+
     sampler.stop()
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": dist.world,
@@ -392,7 +492,7 @@ def run_ours(args, dist: Dist) -> dict:
                    "parallelism": f"dp{dist.world} (independent sequences per rank)"},
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps,
         "clocks": clocks, "decode": dec, "decode_packed": dec_packed,
-        "prefill_other": others or None, "impl": "ours",
+        "prefill_other": others or None, "backward": bwd, "impl": "ours",
     }
     dist.close()
     return res
