@@ -234,6 +234,32 @@ gdn_status gdn_prefill_backward(const void *q, const void *k, const void *v,
                                 float *dbeta, float *dstate_in, void *cuda_stream);
 
 /*
+ * gdn_prefill_backward_static - gdn_prefill_backward with its workspace in
+ * the library's own static device array (64 MiB per device, reserved when
+ * the library's module is loaded) instead of caller memory; it allocates
+ * nothing.  For callers that must not allocate device memory while they
+ * run.  The methods described on the pages have no counterpart: this is an
+ * interface choice.
+ *
+ * Arguments, layouts, outputs and errors as gdn_prefill_backward, without
+ * the workspace.  A call whose workspace would exceed 64 MiB
+ * (gdn_prefill_backward_workspace_bytes) returns GDN_ERR_UNSUPPORTED before
+ * touching the device.  The first call on a device looks up the array's
+ * address (cudaGetSymbolAddress) and fails with GDN_ERR_CUDA if it cannot;
+ * make that first call outside any stream capture.  Calls that overlap on
+ * one device (two streams, or two host threads) share the array and race:
+ * order them.
+ */
+gdn_status gdn_prefill_backward_static(const void *q, const void *k, const void *v,
+                                       const float *g, const float *beta,
+                                       const float *state_in, const int32_t *cu_seqlens,
+                                       int n_seq, int T, int H, int d_k, int d_v,
+                                       gdn_dtype dt, gdn_gate_kind gk, gdn_qdq_mode qdq,
+                                       const void *d_o, const float *dstate_out,
+                                       float *dq, float *dk, float *dv, float *dg,
+                                       float *dbeta, float *dstate_in, void *cuda_stream);
+
+/*
  * gdn_prefill_schedule - which prefill kernel gdn_prefill launches for these
  * shapes on the current device, under the current GDN_PREFILL_CTA_PAIR
  * setting (the same selection code).  Host-only; it may query the device's

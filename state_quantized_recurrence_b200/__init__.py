@@ -23,12 +23,14 @@ from __future__ import annotations
 from ._binding import (  # noqa: F401
     GDN_DTYPE, GDN_GATE, GDN_QDQ, GDN_STATUS, GdnError, check_last_error,
     PackedState, gdn_decode, gdn_decode_into, gdn_decode_packed, gdn_decode_packed_into,
-    gdn_last_error, gdn_prefill, gdn_prefill_backward, gdn_prefill_into, gdn_prefill_schedule,
+    gdn_last_error, gdn_prefill, gdn_prefill_backward, gdn_prefill_backward_static,
+    gdn_prefill_into, gdn_prefill_schedule,
     gdn_state_pack, gdn_state_unpack, lib, library_path, packed_state_empty,
 )
 
 __all__ = [
-    "gdn_prefill", "gdn_prefill_into", "gdn_prefill_backward", "gdn_prefill_schedule",
+    "gdn_prefill", "gdn_prefill_into", "gdn_prefill_backward", "gdn_prefill_backward_static",
+    "gdn_prefill_schedule",
     "gdn_decode", "gdn_decode_into",
     "gdn_decode_packed", "gdn_decode_packed_into", "gdn_state_pack", "gdn_state_unpack",
     "PackedState", "packed_state_empty",

@@ -40,6 +40,8 @@ def _load() -> ctypes.CDLL:
     L.gdn_prefill_backward.argtypes = ([P] * 7 + [I] * 8 + [P, P, P, ctypes.c_size_t]
                                        + [P] * 6 + [P])
     L.gdn_prefill_backward.restype = I
+    L.gdn_prefill_backward_static.argtypes = [P] * 7 + [I] * 8 + [P, P] + [P] * 6 + [P]
+    L.gdn_prefill_backward_static.restype = I
     L.gdn_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, P, P]
     L.gdn_decode.restype = I
     L.gdn_decode_packed.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, P]
@@ -201,6 +203,47 @@ def gdn_prefill_backward(q, k, v, g, beta, d_o, state_in=None, cu_seqlens=None,
         _ptr(dg), _ptr(dbeta), _ptr(dstate_in), _stream(stream))
     if s != 0:
         raise GdnError(s, "gdn_prefill_backward")
+    return dq, dk, dv, dg, dbeta, dstate_in
+
+
+def gdn_prefill_backward_static(q, k, v, g, beta, d_o, state_in=None, cu_seqlens=None,
+                                dstate_out=None, qdq: str = "fp8_tile64", stream=None):
+    """gdn_prefill_backward with the workspace taken from the library's
+    static device array (64 MiB; larger problems raise GDN_ERR_UNSUPPORTED).
+    Calls that overlap on one device share that array: order them.  Returns
+    fp32 ``(dq, dk, dv, dg, dbeta, dstate_in)`` (allocated here with torch)."""
+    _check_dev(q, k, v, g, beta, d_o, state_in, cu_seqlens, dstate_out)
+    _need(q.dim() == 4 and k.shape == q.shape and v.dim() == 4, "q, k, v must be [B, T, H, d]")
+    B, T, H, d_k = q.shape
+    d_v = v.shape[-1]
+    _need(q.dtype in GDN_DTYPE and k.dtype == q.dtype and v.dtype == q.dtype
+          and d_o.dtype == q.dtype and d_o.shape == v.shape, "d_o must be shaped like o, q's dtype")
+    _need(g.dtype == torch.float32 and beta.dtype == torch.float32 and beta.shape == q.shape[:3],
+          "g, beta must be fp32; beta [B, T, H]")
+    gk = _gate_kind(g, 3)
+    _need(g.shape == (q.shape[:3] if gk == "scalar" else q.shape), "g must be [B,T,H] or [B,T,H,d_k]")
+    if cu_seqlens is not None:
+        _need(B == 1 and cu_seqlens.dtype == torch.int32 and cu_seqlens.dim() == 1,
+              "packed layout needs B == 1 and int32 cu_seqlens")
+        n_seq, T_arg = cu_seqlens.numel() - 1, T
+    else:
+        n_seq, T_arg = B, T
+    sshape = (n_seq, H, d_k, d_v)
+    for t in (state_in, dstate_out):
+        _need(t is None or (t.shape == sshape and t.dtype == torch.float32),
+              "states must be fp32 [n_seq, H, d_k, d_v]")
+    f32 = dict(dtype=torch.float32, device=q.device)
+    dq, dk = torch.empty(q.shape, **f32), torch.empty(q.shape, **f32)
+    dv = torch.empty(v.shape, **f32)
+    dg, dbeta = torch.empty(g.shape, **f32), torch.empty(beta.shape, **f32)
+    dstate_in = torch.empty(sshape, **f32)
+    s = lib.gdn_prefill_backward_static(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_in), _ptr(cu_seqlens), n_seq,
+        T_arg, H, d_k, d_v, GDN_DTYPE[q.dtype], GDN_GATE[gk], GDN_QDQ[qdq], _ptr(d_o),
+        _ptr(dstate_out), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg), _ptr(dbeta), _ptr(dstate_in),
+        _stream(stream))
+    if s != 0:
+        raise GdnError(s, "gdn_prefill_backward_static")
     return dq, dk, dv, dg, dbeta, dstate_in
 
 

@@ -616,6 +616,52 @@ gdn_status gdn_prefill_backward(const void *q, const void *k, const void *v, con
 #undef GDN_BQ
 }
 
+}  // extern "C"
+
+namespace {
+// Scratch of gdn_prefill_backward_static: the library's own device memory,
+// reserved with the module on each device that loads it (no per-call
+// allocation).  Every word is written before it is read, so nothing in it
+// needs to start at zero.  Calls that overlap on one device (two streams or
+// host threads) share it and race.
+constexpr size_t kStaticScratchBytes = size_t(64) << 20;
+static __device__ __align__(256) unsigned char g_bwd_scratch[kStaticScratchBytes];
+void *g_bwd_scratch_ptr[kMaxDevices];  // its address per device, looked up once
+}  // namespace
+
+extern "C" {
+
+// For callers that must not allocate device memory while they run (a step
+// whose memory budget is fixed after start-up, where an allocation could
+// fail or stall on the caching allocator): the workspace comes from the
+// static array above instead of the caller.
+gdn_status gdn_prefill_backward_static(const void *q, const void *k, const void *v,
+                                       const float *g, const float *beta, const float *state_in,
+                                       const int32_t *cu_seqlens, int n_seq, int T, int H,
+                                       int d_k, int d_v, gdn_dtype dt, gdn_gate_kind gk,
+                                       gdn_qdq_mode qdq, const void *d_o,
+                                       const float *dstate_out, float *dq, float *dk, float *dv,
+                                       float *dg, float *dbeta, float *dstate_in,
+                                       void *cuda_stream) {
+  const size_t need = gdn_prefill_backward_workspace_bytes(n_seq, T, H, d_k, d_v,
+                                                           cu_seqlens != nullptr);
+  if (need > kStaticScratchBytes) return GDN_ERR_UNSUPPORTED;
+  void *ws = nullptr;
+  if (need > 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return GDN_ERR_CUDA;
+    if (!g_bwd_scratch_ptr[dev]) {
+      void *p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_bwd_scratch) != cudaSuccess || !p) return GDN_ERR_CUDA;
+      g_bwd_scratch_ptr[dev] = p;
+    }
+    ws = g_bwd_scratch_ptr[dev];
+  }
+  return gdn_prefill_backward(q, k, v, g, beta, state_in, cu_seqlens, n_seq, T, H, d_k, d_v, dt,
+                              gk, qdq, d_o, dstate_out, ws, ws ? kStaticScratchBytes : 0, dq, dk,
+                              dv, dg, dbeta, dstate_in, cuda_stream);
+}
+
 int gdn_prefill_schedule(int n_seq, int H, int d_k, int d_v, gdn_dtype dt, gdn_gate_kind gk) {
   if (n_seq < 0 || H <= 0) return -1;
   if ((d_k != 64 && d_k != 128) || (d_v != 64 && d_v != 128)) return -1;

@@ -205,6 +205,19 @@ def test_backward_workspace_and_errors(lib):
     assert bw(lib, n_seq=0) == OK
 
 
+def test_backward_static_rejects_oversize(lib):
+    """A problem whose workspace exceeds the 64 MiB static array is refused
+    before the device is touched."""
+    P, I = ctypes.c_void_p, ctypes.c_int
+    lib.gdn_prefill_backward_static.argtypes = [P] * 7 + [I] * 8 + [P, P] + [P] * 7
+    lib.gdn_prefill_backward_static.restype = I
+    lib.gdn_prefill_backward_workspace_bytes.argtypes = [I] * 6
+    lib.gdn_prefill_backward_workspace_bytes.restype = ctypes.c_size_t
+    assert lib.gdn_prefill_backward_workspace_bytes(4, 4096, 16, 128, 128, 0) > 64 << 20
+    assert lib.gdn_prefill_backward_static(A, A, A, A, A, None, None, 4, 4096, 16, 128, 128, BF16,
+                                           0, 1, A, None, A, A, A, A, A, A, None) == UNSUPPORTED
+
+
 def test_decode_specific_errors(lib):
     assert dc(lib, state=None) == INVALID
     assert dc(lib, state=A + 4) == INVALID
