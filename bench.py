@@ -56,6 +56,7 @@ KERNEL_SOURCES = {
     "prefill_gdn": ["gdn_prefill_pair.cuh", "gdn_tc_util.cuh", "gdn_sm100.cuh", "gdn_common.cuh"],
     "decode": ["gdn_decode.cuh", "gdn_common.cuh"],
     "decode_packed": ["gdn_decode.cuh", "gdn_common.cuh"],
+    "backward": ["gdn_backward.cuh", "gdn_common.cuh"],
 }
 
 
@@ -332,7 +333,8 @@ def measure_backward(args, dist, dev, stream, sampler, peaks, case, steps, warmu
         "kernel": "bwd::prefill_backward_kernel (FFMA, token-reverse with chunk checkpoints)",
         "workspace_bytes": need,
         "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
-                     "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 5), "traffic": None,
+                     "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 5),
+                     "traffic": recorded_traffic("backward"),
                      "bytes_per_launch": nbytes, "peak_source": peaks["source"]},
         "gpu_launches": steps, "clocks": sampler.summary(t_wall0, t_wall1),
     }
@@ -428,6 +430,13 @@ def run_ours(args, dist: Dist) -> dict:
     stream = torch.cuda.current_stream(dev)
     sampler = ClockSampler(dist.local)
 
+    if args.only == "backward":  # profiler captures of the backward kernel
+        bwd = measure_backward(args, dist, dev, stream, sampler, peaks,
+                               gs.CONFIGS["gdn_prefill"], args.steps, args.warmup)
+        sampler.stop()
+        dist.close()
+        return {"metric": bwd["metric"], "value": bwd["value"], "unit": bwd["unit"],
+                "n_gpus": dist.world, "impl": "ours", "backward": bwd}
     if args.only in ("decode", "decode_packed"):  # profiler captures of one decode kernel
         dec = run_decode(args, dist, dev, stream, sampler, peaks, packed=args.only == "decode_packed")
         sampler.stop()
@@ -672,7 +681,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-decode", action="store_true")
-    ap.add_argument("--only", choices=["prefill", "decode", "decode_packed"], default=None,
+    ap.add_argument("--only", choices=["prefill", "decode", "decode_packed", "backward"],
+                    default=None,
                     help="measure one kernel only (profiler captures)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-others", action="store_true",
