@@ -431,8 +431,11 @@ def run_ours(args, dist: Dist) -> dict:
     sampler = ClockSampler(dist.local)
 
     if args.only == "backward":  # profiler captures of the backward kernel
-        bwd = measure_backward(args, dist, dev, stream, sampler, peaks,
-                               gs.CONFIGS["gdn_prefill"], args.steps, args.warmup)
+        bcase = gs.CONFIGS["gdn_prefill"]
+        if args.small:  # the same 128 CTAs, 4 chunks each
+            bcase = gs.small_case("gdn_prefill", T=256)
+        bwd = measure_backward(args, dist, dev, stream, sampler, peaks, bcase, args.steps,
+                               args.warmup)
         sampler.stop()
         dist.close()
         return {"metric": bwd["metric"], "value": bwd["value"], "unit": bwd["unit"],

@@ -20,6 +20,7 @@
 // workspace; phase 2 walks the chunks backwards: it recomputes the chunk's
 // per-token states into the workspace, then runs the reverse recurrence
 // over them.  Every thread reads back only the workspace words it wrote.
+// Each token's inputs are fetched into registers one token ahead.
 // Sums over value columns (dq, dk, dg, dbeta) come from one atomic add per
 // tile into zeroed fp32 buffers, so with at most two tiles (d_v <= 128)
 // the result does not depend on the order of the adds.
@@ -177,20 +178,37 @@ prefill_backward_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
   auto chunk_ws = [&](int c) { return ws_chunk + (((slot0 + c) * H + h) * nvt + vt) * (long long)TILE; };
   float *tok_ws = ws_tok + (long long)blockIdx.x * kChunk * TILE;
 
-  // inputs of one token: k, q, per-key decays in shared memory; the rest in
-  // registers
+  // Inputs of one token, fetched into registers one token ahead and then
+  // committed: k, q and the per-key decays to shared memory, the rest to
+  // registers.
+  struct Raw {
+    float kf, qf, gf, gs, bt;
+    float4 v4, do4;
+  };
+  auto fetch = [&](long long tok, bool with_do, Raw &r) {
+    if (tid < DK) {
+      r.kf = to_f32(k[(tok * H + h) * DK + tid]);
+      r.qf = to_f32(q[(tok * H + h) * DK + tid]);
+      if (PER_KEY) r.gf = __ldg(g + (tok * H + h) * DK + tid);
+    }
+    if (!PER_KEY) r.gs = __ldg(g + tok * H + h);
+    r.bt = __ldg(beta + tok * H + h);
+    r.v4 = load4(v + (tok * H + h) * DV + col);
+    if (with_do) r.do4 = load4(dout + (tok * H + h) * DV + col);
+  };
   float al_s = 1.0f, bt = 0.0f;
   float4 v4, do4;
-  auto stage = [&](long long tok) {
+  auto commit = [&](const Raw &r) {
     __syncthreads();  // the previous token's shared inputs have been read
     if (tid < DK) {
-      s_k[tid] = to_f32(k[(tok * H + h) * DK + tid]);
-      s_q[tid] = to_f32(q[(tok * H + h) * DK + tid]);
-      if (PER_KEY) s_al[tid] = expf(__ldg(g + (tok * H + h) * DK + tid));
+      s_k[tid] = r.kf;
+      s_q[tid] = r.qf;
+      if (PER_KEY) s_al[tid] = expf(r.gf);
     }
-    if (!PER_KEY) al_s = expf(__ldg(g + tok * H + h));
-    bt = __ldg(beta + tok * H + h);
-    v4 = load4(v + (tok * H + h) * DV + col);
+    if (!PER_KEY) al_s = expf(r.gs);
+    bt = r.bt;
+    v4 = r.v4;
+    do4 = r.do4;
     __syncthreads();
   };
   // forward token step on the slab: h <- diag(alpha) h + k u^T; returns a
@@ -217,20 +235,22 @@ prefill_backward_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
   };
 
   float4 hst[RPT], htd[RPT];
+  Raw cur, nxt;
+  cur.do4 = nxt.do4 = make_float4(0.f, 0.f, 0.f, 0.f);
   // ---- phase 1: forward with the chunk-end QDQ; chunk-start states kept ----
 #pragma unroll
   for (int j = 0; j < RPT; ++j) {
     hst[j] = make_float4(0.f, 0.f, 0.f, 0.f);
     if (state_in) hst[j] = *reinterpret_cast<const float4 *>(state_in + st_off + (rg + 16 * j) * DV + col);
   }
-  for (int c = 0; c < n_chunks; ++c) {
-    ws_store<RPT>(chunk_ws(c), tid, hst);
-    const int n = (int)min((long long)kChunk, L - (long long)c * kChunk);
-    for (int t = 0; t < n; ++t) {
-      stage(t0 + (long long)c * kChunk + t);
-      (void)fwd_step(hst, htd);
-    }
-    qdq_slab<RPT, QK, GROUP>(hst, red8, warp, lane);  // (only the starts are kept)
+  if (L > 0) fetch(t0, false, cur);
+  for (long long t = 0; t < L; ++t) {
+    if (t % kChunk == 0) ws_store<RPT>(chunk_ws((int)(t / kChunk)), tid, hst);
+    commit(cur);
+    if (t + 1 < L) fetch(t0 + t + 1, false, nxt);
+    (void)fwd_step(hst, htd);
+    if (t % kChunk == kChunk - 1 || t == L - 1) qdq_slab<RPT, QK, GROUP>(hst, red8, warp, lane);
+    cur = nxt;
   }
 
   // ---- phase 2: chunks in reverse ----
@@ -244,17 +264,21 @@ prefill_backward_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
     const int n = (int)min((long long)kChunk, L - (long long)c * kChunk);
     const long long tb = t0 + (long long)c * kChunk;
     ws_load<RPT>(chunk_ws(c), tid, hst);
+    fetch(tb, false, cur);
     for (int t = 0; t < n; ++t) {  // per-token states H_{t-1}
       ws_store<RPT>(tok_ws + (long long)t * TILE, tid, hst);
-      stage(tb + t);
+      commit(cur);
+      if (t + 1 < n) fetch(tb + t + 1, false, nxt);
       (void)fwd_step(hst, htd);
+      cur = nxt;
     }
+    fetch(tb + n - 1, true, cur);
     for (int t = n - 1; t >= 0; --t) {
       const long long tok = tb + t;
       float4 hp[RPT];
       ws_load<RPT>(tok_ws + (long long)t * TILE, tid, hp);
-      stage(tok);
-      do4 = load4(dout + (tok * H + h) * DV + col);
+      commit(cur);
+      if (t > 0) fetch(tok - 1, true, nxt);
 #pragma unroll
       for (int j = 0; j < RPT; ++j) hst[j] = hp[j];
       const float4 a = fwd_step(hst, htd);  // hst = Hn, htd = Ht
@@ -311,6 +335,7 @@ prefill_backward_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
         const float tot = sum_block(galpha, red8, warp, lane);
         if (tid == 0) atomicAdd(dg + tok * H + h, al_s * tot);
       }
+      cur = nxt;
     }
   }
 #pragma unroll
