@@ -246,15 +246,16 @@ gdn_status make_token_map(CUtensorMap *m, const void *ptr, int H, long long rows
 
 template <int QK, int GR>
 gdn_status launch_tc_one(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
-                         const float *g, const float *beta, const float *state_in,
+                         const CUtensorMap &mo, const float *g, const float *beta,
+                         const float *state_in,
                          const int32_t *cu, int T, int H, float scale, __nv_bfloat16 *o,
                          float *state_out, unsigned *err, unsigned blocks, cudaStream_t st) {
   auto kern = gdn::tc::prefill_tc_kernel<QK, GR>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)gdn::tc::kSmemBytes) != cudaSuccess)
     return GDN_ERR_CUDA;
-  kern<<<blocks, gdn::tc::kThreads, gdn::tc::kSmemBytes, st>>>(mq, mk, mv, g, beta, state_in, cu,
-                                                               T, H, scale, o, state_out, err);
+  kern<<<blocks, gdn::tc::kThreads, gdn::tc::kSmemBytes, st>>>(mq, mk, mv, mo, g, beta, state_in,
+                                                               cu, T, H, scale, o, state_out, err);
   return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
@@ -340,10 +341,10 @@ gdn_status launch_prefill_tc(const void *q, const void *k, const void *v, const 
   const float scale = (float)(1.0 / sqrt(128.0));
   __nv_bfloat16 *oo = static_cast<__nv_bfloat16 *>(o);
   const unsigned nb = (unsigned)blocks;
+  CUtensorMap mo;  // outputs [rows, H, 128] bf16, stored by whole 64-token chunks
+  if ((s = make_token_map(&mo, o, H, rows, true)) != GDN_OK) return s;
   if (use_pair(blocks)) {
     if (blocks > 0x3fffffffLL) return GDN_ERR_UNSUPPORTED;
-    CUtensorMap mo;  // outputs [rows, H, 128] bf16, stored by whole 64-token chunks
-    if ((s = make_token_map(&mo, o, H, rows, true)) != GDN_OK) return s;
 #define GDN_TP(QK, GR) \
   launch_pair_one<QK, GR>(mq, mk, mv, mo, g, beta, state_in, cu, T, H, scale, oo, state_out, err, nb, st)
     if (kind == gdn::kQdqNone) return GDN_TP(gdn::kQdqNone, 32);
@@ -354,7 +355,7 @@ gdn_status launch_prefill_tc(const void *q, const void *k, const void *v, const 
 #undef GDN_TP
   }
 #define GDN_TC(QK, GR) \
-  launch_tc_one<QK, GR>(mq, mk, mv, g, beta, state_in, cu, T, H, scale, oo, state_out, err, nb, st)
+  launch_tc_one<QK, GR>(mq, mk, mv, mo, g, beta, state_in, cu, T, H, scale, oo, state_out, err, nb, st)
   if (kind == gdn::kQdqNone) return GDN_TC(gdn::kQdqNone, 32);
   if (kind == gdn::kQdqFp8Tile) return GDN_TC(gdn::kQdqFp8Tile, 32);
   if (group == 16) return GDN_TC(gdn::kQdqInt8, 16);

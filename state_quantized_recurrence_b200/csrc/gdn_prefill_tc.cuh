@@ -63,6 +63,12 @@ constexpr int LDT = 68;                 // fp32 row stride of the solve's matric
 constexpr uint32_t OFF_P = 188416;      // solve partial products fp32 [32 x LDT]
 constexpr uint32_t OFF_T = OFF_P + 32 * LDT * 4;  // solve T fp32 [64 x LDT]
 constexpr uint32_t OFF_SMALL = OFF_T + 64 * LDT * 4;  // gates, flags, barriers
+// Output tile of a whole chunk, bf16 [v half][64 t][64 v], 128B-swizzled, for
+// the TMA store: it borrows the solve's scratch (P, T), which is idle from
+// epilogue 4 until the next chunk's solve.
+constexpr uint32_t OFF_O = OFF_P;
+static_assert(OFF_O % 1024 == 0 && OFF_O + 16384 <= OFF_SMALL, "output tile");
+constexpr int kStoreTid = 224;
 constexpr uint32_t kSmemBytes = OFF_SMALL + 4096 + 1024;  // + alignment slack
 // Region X: first half of a chunk: A fp32 [64 x LDT] at [0, 17408) (its last
 // row overlaps T hi, which is written only after the solve has read A), T hi
@@ -139,7 +145,8 @@ __device__ __forceinline__ void convert_kq(uint8_t *buf, int n, int t, int nthr)
 template <int QK, int GROUP>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ g,
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                  const float *__restrict__ g,
                   const float *__restrict__ beta, const float *__restrict__ state_in,
                   const int *__restrict__ cu_seqlens, int T, int H, float scale,
                   __nv_bfloat16 *__restrict__ o, float *__restrict__ state_out,
@@ -397,6 +404,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       }
     }
     sm100::fence_proxy_async();
+    // the previous chunk's output tile (in the solve's scratch) has been read
+    if (tid == kStoreTid) sm100::bulk_wait_read_all();
     __syncthreads();
     if (sm->abort) break;
 
@@ -634,7 +643,46 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     {
       // O^T[v][t] = scale (gamma_t (Q H0)^T[v][t] + (Aqk Vn)^T[v][t]) ->
       // o[t][h][v]: warpgroup wg writes tokens 32 wg .. + 31
-      {
+      if (n == kC) {
+        // a whole chunk: fragments of 16 value rows x 32 tokens, packed to
+        // bf16 token pairs and stored transposed into the output tile; the TMA
+        // store is issued after the barrier that ends this chunk
+        const int c = lane & 3;
+        const float sh = scale * hsv;
+#pragma unroll
+        for (int hl = 0; hl < 2; ++hl) {
+          const int L = 32 * (warp & 3) + 16 * hl;  // first value row of the block
+          const uint32_t lsel = (uint32_t)L << 16;
+          uint32_t qh[16], av[16];
+          sm100::tmem_ld16x256b_x4(tmem + lsel + TM_D2 + 64 + 32 * wg, qh);
+          sm100::tmem_ld16x256b_x4(tmem + lsel + TM_D5 + 32 * wg, av);
+          uint32_t pk[8];
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const float2 g2 = *reinterpret_cast<const float2 *>(gt->gam + 32 * wg + 8 * kk + 2 * c);
+            const float s0 = sh * g2.x, s1 = sh * g2.y;
+#pragma unroll
+            for (int hv = 0; hv < 2; ++hv) {  // value rows L + lane / 4 and L + 8 + lane / 4
+              const int e = 4 * kk + 2 * hv;
+              const float o0 = fmaf(s0, __uint_as_float(qh[e]), scale * __uint_as_float(av[e]));
+              const float o1 = fmaf(s1, __uint_as_float(qh[e + 1]), scale * __uint_as_float(av[e + 1]));
+              __nv_bfloat162 p2 = __floats2bfloat162_rn(o0, o1);
+              pk[2 * kk + hv] = *reinterpret_cast<uint32_t *>(&p2);
+            }
+          }
+#pragma unroll
+          for (int k0 = 0; k0 < 4; k0 += 2) {
+            const int m = lane >> 3, rr = lane & 7;
+            const int t = 32 * wg + 8 * (k0 + (m >> 1)) + rr;
+            const int v0 = L + 8 * (m & 1);
+            const uint32_t addr = base + OFF_O + (uint32_t)(v0 >> 6) * 8192u + (uint32_t)t * 128u +
+                                  ((uint32_t)(((v0 & 63) >> 3) ^ (t & 7)) << 4);
+            sm100::stmatrix_x4_trans(addr, pk[2 * k0], pk[2 * k0 + 1], pk[2 * k0 + 2],
+                                     pk[2 * k0 + 3]);
+          }
+        }
+        op_dst = nullptr;
+      } else {  // a partial last chunk: stored directly after the loop
         float qh[32], av[32];
         sm100::tmem_ld32(tmem + lane_off + TM_D2 + 64 + 32 * wg, qh);
         sm100::tmem_ld32(tmem + lane_off + TM_D5 + 32 * wg, av);
@@ -745,11 +793,17 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     sm100::fence_proxy_async();
     sm100::tc_fence_before();
     __syncthreads();
+    if (tid == kStoreTid && n == kC) {
+      sm100::tma_store_3d(&tm_o, gbase + OFF_O, 0, h, (int)tb);
+      sm100::tma_store_3d(&tm_o, gbase + OFF_O + 8192, 64, h, (int)tb);
+      sm100::bulk_commit();
+    }
     if (tid == 0) sm->exact = QK == kQdqFp8Tile ? 1 : 0;
     __syncthreads();
   }
 
-  flush_outputs();  // the last chunk's outputs
+  flush_outputs();  // a partial last chunk's outputs
+  if (tid == kStoreTid) sm100::bulk_wait_all();
 
   // An aborted CTA lets its outstanding TMA loads land (again bounded)
   // before its shared memory is released.
