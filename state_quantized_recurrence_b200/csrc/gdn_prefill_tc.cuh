@@ -19,8 +19,9 @@
 // key axis): [K;Q] K^T, H0^T [K;Q]^T, R^T T^T, Vn^T Aqk^T and K^T (dVn).  The
 // A operands R^T and Vn^T go to TMEM (their epilogue thread already owns the
 // row); the rest are fp16 in 128-byte-swizzled shared-memory tiles.  q/k
-// arrive by TMA (bf16, swizzled) into a double buffer and are converted to
-// fp16 in place (exact for |x| in the fp16 range).  Non-exact fp32 operands
+// arrive by TMA (bf16, swizzled) into a double buffer; [K;Q] K^T reads the
+// raw bf16 tile, which is then converted to fp16 in place for the state
+// products (exact for |x| in the fp16 range).  Non-exact fp32 operands
 // (H0, R, T, dVn) are split into hi + lo fp16 pairs (about 22 significant
 // bits); with FP8 QDQ the state after the first boundary is exactly
 // E4M3 code x tile scale, so H0 enters as one exact fp16 term and the scale
@@ -29,13 +30,18 @@
 // Schedule of one chunk c (256 threads, warpgroups WG0 = warps 0-3 and
 // WG1 = warps 4-7, both covering TMEM lanes 0-127):
 //   MMA2(c)                       [thread 0]
-//   WG0: A, Aqk from MMA1(c); triangular solve; T hi/lo
-//   WG1: R = beta (V - gamma P) -> TMEM; next gates; convert chunk c+1's
-//        [K;Q] in place and issue MMA1(c+1)
-//   MMA3(c): Vn^T = R^T T^T       [thread 0]
+//   all: A, Aqk from MMA1(c)
+//   WG0: triangular solve, levels 16 and 32
+//   WG1: R = beta (V - gamma P) -> TMEM; next gates; MMA1(c+1) on the next
+//        chunk's raw bf16 tile
+//   all: the solve's last level and T hi/lo
+//   MMA3(c): Vn^T = R^T T^T       [thread 0]; meanwhile half of the next
+//        tile's in-place fp16 conversion (once MMA1(c+1) has read it)
 //   all: Vn^T -> TMEM, dVn^T hi/lo -> shared memory
-//   MMA4(c): (Aqk Vn)^T, MMA5(c): H += K^T dVn   [thread 0]
-//   all: outputs, state QDQ (each warpgroup one 64-column tile), H0 operands;
+//   MMA4(c): (Aqk Vn)^T, MMA5(c): H += K^T dVn   [thread 0]; meanwhile the
+//        other half of the conversion
+//   all: outputs (a whole chunk's through a swizzled tile and TMA stores),
+//        state QDQ (each warpgroup one 64-column tile), H0 operands;
 //        prefetch chunk c+2 into the buffer chunk c released
 // Every mbarrier wait is bounded; on a timeout the CTA records kErrTimeout,
 // stops, lets its in-flight TMA loads land, releases its TMEM and returns.
@@ -108,38 +114,6 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, Sm
     return false;
   }
   return true;
-}
-
-// In-place bf16 -> fp16 conversion of one [K;Q] buffer (16-byte chunks in
-// their swizzled positions); rows of tokens past n are zeroed.  `nthr`
-// threads (a multiple of 128), this one being `t`.  Plain shared-memory
-// accesses in batches of four independent chunks, so the loads of a batch
-// are in flight together.
-__device__ __forceinline__ void convert_kq(uint8_t *buf, int n, int t, int nthr) {
-  for (int e0 = t; e0 < 2048; e0 += 4 * nthr) {
-    uint4 x[4];
-    uint8_t *ad[4];
-    bool live[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int e = e0 + u * nthr;  // < 2048: 2048 is a multiple of 4 * nthr
-      const int blk = e >> 10, rw = (e >> 3) & 127, ch = e & 7;
-      ad[u] = buf + blk * 16384 + rw * 128 + ch * 16;
-      live[u] = (rw & 63) < n;
-      x[u] = *reinterpret_cast<const uint4 *>(ad[u]);
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const uint32_t in[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
-      uint32_t w[4] = {0u, 0u, 0u, 0u};
-      if (live[u]) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          w[j] = pack_h2(__uint_as_float(in[j] << 16), __uint_as_float(in[j] & 0xffff0000u));
-      }
-      *reinterpret_cast<uint4 *>(ad[u]) = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-  }
 }
 
 template <int QK, int GROUP>
@@ -237,7 +211,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     sm->v_pend = 1 + (j & 1);
   };
 
-  const uint32_t ID_KQ = sm100::idesc_f16_f32(128, 64, 0, 0);
+  // [K;Q] K^T on the raw bf16 tile (exact products), before its conversion
+  const uint32_t ID_KQ = sm100::idesc_f16_f32(128, 64, 0, 0) | (1u << 7) | (1u << 10);
   const uint32_t ID_H2 = sm100::idesc_f16_f32(128, 128, 1, 0);
   const uint32_t ID_H2LO = sm100::idesc_f16_f32(128, 64, 1, 0);
   const uint32_t ID_64 = sm100::idesc_f16_f32(128, 64, 0, 0);
@@ -287,17 +262,20 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       sm100::tmem_st32(tmem + lane_off + TM_D4 + c0, x);
     }
   }
-  // ---- chunk 0's [K;Q]: wait, convert, MMA1 (later chunks' are prepared
-  //      during the previous chunk) ----
+  // ---- chunk 0's [K;Q]: wait, MMA1 on the raw tile, then convert it for
+  //      MMAs 2 and 5 (later chunks' during the previous chunk) ----
   if (wait_or_abort(&sm->bar_qk[0], 0, sm, err) && tid == 0) sm->qk_pend[0] = 0;
-  convert_kq(gbase + OFF_KQ, (int)min((long long)kC, L), tid, kThreads);
-  sm100::fence_proxy_async();
-  sm100::tc_fence_before();
   __syncthreads();
   if (warp == 0 && !sm->abort) {
     sm100::tc_fence_after();
     issue_mma1(0);
   }
+  wait_or_abort(&sm->bar_m1, 0, sm, err);
+  convert_kq_half(gbase + OFF_KQ, (int)min((long long)kC, L), tid, 0);
+  convert_kq_half(gbase + OFF_KQ, (int)min((long long)kC, L), tid, 1);
+  sm100::fence_proxy_async();
+  sm100::tc_fence_before();
+  __syncthreads();
 
   // Outputs of a chunk are computed in its last epilogue but stored at the
   // start of the next chunk (or after the loop), off the state path: 32
@@ -466,55 +444,6 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         *reinterpret_cast<float4 *>(sT + (r0 + rr) * LDT + c0b + cc) =
             make_float4(-q.x, -q.y, -q.z, -q.w);
       }
-      asm volatile("bar.sync 3, 128;" ::: "memory");
-      // Level 2: the lower-left 32x32 block: T_21 = -T_22 (A_21 T_11).
-      {
-        const int rr = tid >> 2, cc = (tid & 3) * 8;
-        const float *arow = sA + (32 + rr) * LDT;
-        const float *tcol = sT + cc;
-        float p[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int m = 0; m < 32; ++m) {
-          const float a = arow[m];
-          const float4 t0v = *reinterpret_cast<const float4 *>(tcol + m * LDT);
-          const float4 t1v = *reinterpret_cast<const float4 *>(tcol + m * LDT + 4);
-          p[0] += a * t0v.x; p[1] += a * t0v.y; p[2] += a * t0v.z; p[3] += a * t0v.w;
-          p[4] += a * t1v.x; p[5] += a * t1v.y; p[6] += a * t1v.z; p[7] += a * t1v.w;
-        }
-        *reinterpret_cast<float4 *>(sP + rr * LDT + cc) = make_float4(p[0], p[1], p[2], p[3]);
-        *reinterpret_cast<float4 *>(sP + rr * LDT + cc + 4) = make_float4(p[4], p[5], p[6], p[7]);
-        asm volatile("bar.sync 3, 128;" ::: "memory");
-        const float *trow = sT + (32 + rr) * LDT + 32;
-        const float *pcol = sP + cc;
-        float q[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int m = 0; m < 32; ++m) {
-          const float t = trow[m];
-          const float4 p0v = *reinterpret_cast<const float4 *>(pcol + m * LDT);
-          const float4 p1v = *reinterpret_cast<const float4 *>(pcol + m * LDT + 4);
-          q[0] += t * p0v.x; q[1] += t * p0v.y; q[2] += t * p0v.z; q[3] += t * p0v.w;
-          q[4] += t * p1v.x; q[5] += t * p1v.y; q[6] += t * p1v.z; q[7] += t * p1v.w;
-        }
-        float *tout = sT + (32 + rr) * LDT + cc;
-        *reinterpret_cast<float4 *>(tout) = make_float4(-q[0], -q[1], -q[2], -q[3]);
-        *reinterpret_cast<float4 *>(tout + 4) = make_float4(-q[4], -q[5], -q[6], -q[7]);
-      }
-      asm volatile("bar.sync 3, 128;" ::: "memory");
-      // T -> hi/lo fp16 tiles [tok][tok'] (upper triangle zero).
-      {
-        const int r = tid >> 1, cpart = (tid & 1) * 32;
-        const float *trow = sT + r * LDT + cpart;
-        float x[32];
-#pragma unroll
-        for (int i = 0; i < 32; i += 4) {
-          const float4 t4 = *reinterpret_cast<const float4 *>(trow + i);
-          x[i] = cpart + i <= r ? t4.x : 0.f;
-          x[i + 1] = cpart + i + 1 <= r ? t4.y : 0.f;
-          x[i + 2] = cpart + i + 2 <= r ? t4.z : 0.f;
-          x[i + 3] = cpart + i + 3 <= r ? t4.w : 0.f;
-        }
-        store32_hl(base + OFF_X + X_THI, base + OFF_X + X_TLO, r, cpart >> 3, x);
-      }
     } else {
       // ---- WG1, epilogue 2: R = diag(beta) (V - diag(gamma) P) -> TMEM as
       //      the A operand of MMA 3; then the next chunk's gates (warp 7) ----
@@ -555,21 +484,69 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         sm100::tmem_st16(tmem + lane_off + TM_RLO + 16 * half, wlo);
       }
       if (warp == 7 && !last) finish_gates(gt_next, graw, (int)min((long long)kC, L - c0 - kC), lane);
-      if (!last) {
-        // Still inside WG0's solve: prepare the next chunk - convert its
-        // [K;Q] (landed by TMA a chunk ago) and issue its MMA 1 (D1 was read
-        // by epilogue 1 already).
+      if (!last && warp == 4) {
+        // the next chunk's MMA 1 on its raw tile (landed by TMA a chunk ago;
+        // D1 was read by epilogue 1 already); the tile is converted later
         const int nb = kb ^ 1;
-        if (wait_or_abort(&sm->bar_qk[nb], (uint32_t)(((it + 1) >> 1) & 1), sm, err) && tid == 128)
-          sm->qk_pend[nb] = 0;
-        convert_kq(gbase + OFF_KQ + nb * 32768, (int)min((long long)kC, L - c0 - kC),
-                   tid - 128, 128);
-        sm100::fence_proxy_async();
-        asm volatile("bar.sync 4, 128;" ::: "memory");
-        if (warp == 4 && !sm->abort) {
-          sm100::tc_fence_after();
-          issue_mma1(nb);
-        }
+        const bool ok = __all_sync(
+            0xffffffffu,
+            wait_or_abort(&sm->bar_qk[nb], (uint32_t)(((it + 1) >> 1) & 1), sm, err));
+        if (ok && lane == 0) sm->qk_pend[nb] = 0;
+        sm100::tc_fence_after();
+        if (__all_sync(0xffffffffu, ok && !sm->abort)) issue_mma1(nb);
+      }
+    }
+    __syncthreads();  // T11, T22 and the level-0 blocks final; R in TMEM
+    // Level 2 (all warps): the lower-left 32x32 block T_21 = -T_22 (A_21 T_11),
+    // each thread 4 entries of P = A_21 T_11, then of T_21 = -T_22 P
+    {
+      const int rr = tid >> 3, cc = (tid & 7) * 4;
+      const float *arow = sA + (32 + rr) * LDT;
+      const float *tcol = sT + cc;
+      float4 p = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int m = 0; m < 32; ++m) {
+        const float a = arow[m];
+        const float4 t4 = *reinterpret_cast<const float4 *>(tcol + m * LDT);
+        p.x += a * t4.x; p.y += a * t4.y; p.z += a * t4.z; p.w += a * t4.w;
+      }
+      *reinterpret_cast<float4 *>(sP + rr * LDT + cc) = p;
+      __syncthreads();
+      const float *trow = sT + (32 + rr) * LDT + 32;
+      const float *pcol = sP + cc;
+      float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int m = 0; m < 32; ++m) {
+        const float t = trow[m];
+        const float4 p4 = *reinterpret_cast<const float4 *>(pcol + m * LDT);
+        q.x += t * p4.x; q.y += t * p4.y; q.z += t * p4.z; q.w += t * p4.w;
+      }
+      *reinterpret_cast<float4 *>(sT + (32 + rr) * LDT + cc) = make_float4(-q.x, -q.y, -q.z, -q.w);
+    }
+    __syncthreads();
+    // T -> hi/lo fp16 tiles [tok][tok'] (upper triangle zero), all warps:
+    // row tid / 4, columns 16 (tid % 4) .. + 15
+    {
+      const int r = tid >> 2, cpart = (tid & 3) * 16;
+      const float *trow = sT + r * LDT + cpart;
+      float x[16];
+#pragma unroll
+      for (int i = 0; i < 16; i += 4) {
+        const float4 t4 = *reinterpret_cast<const float4 *>(trow + i);
+        x[i] = cpart + i <= r ? t4.x : 0.f;
+        x[i + 1] = cpart + i + 1 <= r ? t4.y : 0.f;
+        x[i + 2] = cpart + i + 2 <= r ? t4.z : 0.f;
+        x[i + 3] = cpart + i + 3 <= r ? t4.w : 0.f;
+      }
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t h0, h1, h2, h3, l0, l1, l2, l3;
+        split_h2(x[8 * c], x[8 * c + 1], h0, l0);
+        split_h2(x[8 * c + 2], x[8 * c + 3], h1, l1);
+        split_h2(x[8 * c + 4], x[8 * c + 5], h2, l2);
+        split_h2(x[8 * c + 6], x[8 * c + 7], h3, l3);
+        st_shared_v4(sw128(base + OFF_X + X_THI, r, (cpart >> 3) + c), h0, h1, h2, h3);
+        st_shared_v4(sw128(base + OFF_X + X_TLO, r, (cpart >> 3) + c), l0, l1, l2, l3);
       }
     }
     sm100::fence_proxy_async();
@@ -594,6 +571,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         sm100::mma_commit(&sm->bar_m3);
       }
       __syncwarp();
+    }
+    // while MMA 3 runs: once the next chunk's MMA 1 has read its raw tile,
+    // the first half of the tile's conversion (for its MMAs 2 and 5)
+    if (!last) {
+      wait_or_abort(&sm->bar_m1, (uint32_t)((it + 1) & 1), sm, err);
+      convert_kq_half(gbase + OFF_KQ + (kb ^ 1) * 32768, (int)min((long long)kC, L - c0 - kC),
+                      tid, 0);
     }
 
     // ---- epilogue 3: Vn^T hi -> TMEM (A of MMA 4); decayed dVn^T hi/lo -> smem ----
@@ -634,6 +618,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       }
       __syncwarp();
     }
+    // while MMAs 4 and 5 run: the second half of the conversion
+    if (!last)
+      convert_kq_half(gbase + OFF_KQ + (kb ^ 1) * 32768, (int)min((long long)kC, L - c0 - kC),
+                      tid, 1);
 
     // ---- epilogue 4 ----
     wait_or_abort(&sm->bar_m4, par, sm, err);

@@ -111,6 +111,35 @@ __device__ __forceinline__ uint32_t fp8_code_pair(float x0, float x1, float s2, 
   return *reinterpret_cast<const uint32_t *>(&hh);
 }
 
+// In-place bf16 -> fp16 conversion of half `part` (the key columns
+// 64 part .. + 63) of one [K;Q] buffer by 256 threads, this one being `t`:
+// 1024 16-byte chunks in their swizzled positions, four per thread with the
+// loads in flight together; rows of tokens past n are zeroed.
+__device__ __forceinline__ void convert_kq_half(uint8_t *buf, int n, int t, int part) {
+  uint4 x[4];
+  uint8_t *ad[4];
+  bool live[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int e = u * 256 + t;  // < 1024
+    const int rw = e >> 3, ch = e & 7;
+    ad[u] = buf + part * 16384 + rw * 128 + ch * 16;
+    live[u] = (rw & 63) < n;
+    x[u] = *reinterpret_cast<const uint4 *>(ad[u]);
+  }
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const uint32_t in[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
+    uint32_t w[4] = {0u, 0u, 0u, 0u};
+    if (live[u]) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        w[j] = pack_h2(__uint_as_float(in[j] << 16), __uint_as_float(in[j] & 0xffff0000u));
+    }
+    *reinterpret_cast<uint4 *>(ad[u]) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
 __device__ __forceinline__ uint64_t kdesc(uint32_t addr) {
   return sm100::smem_desc_sw128(addr, 16, 1024);
 }
