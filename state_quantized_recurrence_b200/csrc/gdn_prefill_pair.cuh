@@ -31,8 +31,8 @@
 //
 // Off the chain CTA's critical path, in the windows where its warps would
 // wait for the tensor cores: the in-place fp16 conversion of the next [K;Q]
-// tile (one half while MMA 2 runs, one while MMAs 4 and 5 run), and the
-// previous chunk's outputs with the next chunk's gates (while MMA 3 runs).
+// tile (one half while MMA 2 runs, one with the next chunk's gates while
+// MMA 3 runs), and the previous chunk's outputs (while MMAs 4 and 5 run).
 // Outputs leave by TMA stores of a staged 64-token tile.
 //
 // Hand-off: the copy completes its bytes on the chain CTA's `rx_full`
@@ -541,8 +541,8 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     __syncthreads();
 
     // Outputs of chunk j: O^T[v][t] = scale (gamma_t hs_j (Q H0)^T[v][t] +
-    // (Aqk Vn)^T[v][t]) -> o[t][h][v].  Run during chunk j+1's MMA 3, off the
-    // state chain; warpgroup wg covers tokens 32 wg .. + 31.  A whole chunk
+    // (Aqk Vn)^T[v][t]) -> o[t][h][v].  Run during chunk j+1's MMAs 4 and 5,
+    // off the state chain; warpgroup wg covers tokens 32 wg .. + 31.  A whole chunk
     // goes through a shared-memory tile and two TMA stores issued by thread
     // 224; a partial chunk (the last of a sequence) is stored directly, so
     // that no row of the neighbouring sequence is written.
@@ -718,13 +718,12 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
         __syncwarp();
       }
-      // while MMA 3 runs: the previous chunk's outputs (its MMA 4 is complete,
-      // and this chunk's MMA 4 is issued only after the barrier below)
-      if (it > 0) out_epilogue(it - 1, tb_prev, n_prev, hs_prev);
-      // and the next chunk's gates (slot (it+1) % 3 was last read by the
-      // output epilogue of chunk it-2), visible to epilogue 4 after the
-      // barrier that follows epilogue 3
+      // while MMA 3 runs: the next chunk's gates (slot (it+1) % 3 was last
+      // read by the output epilogue of chunk it-2), visible to epilogue 4
+      // after the barrier that follows epilogue 3, and the second half of
+      // the next chunk's conversion
       if (warp == 7 && !last) finish_gates(gt_next, graw, chunk_len(it + 1), lane);
+      if (!last) convert_kq_half(gbase + C_KQ + nb * 32768, chunk_len(it + 1), tid, 1);
 
       // ---- epilogue 3: Vn^T hi -> TMEM (A of MMA 4); decayed dVn^T hi/lo -> smem ----
       {
@@ -764,8 +763,9 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
         __syncwarp();
       }
-      // while MMAs 4 and 5 run: the second half of the next chunk's conversion
-      if (!last) convert_kq_half(gbase + C_KQ + nb * 32768, chunk_len(it + 1), tid, 1);
+      // while MMAs 4 and 5 run: the previous chunk's outputs (its MMA 4 wrote
+      // the other TMEM region; its output tile was read out a chunk ago)
+      if (it > 0) out_epilogue(it - 1, tb_prev, n_prev, hs_prev);
 
       // ---- epilogue 4 ----
       wait_local(&sm->bar_m4, par, sm, err);
