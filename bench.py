@@ -220,9 +220,20 @@ class Dist:
 
 
 # ------------------------------------------------------------ our arm
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_baseline_prefill(case, inp, max_seconds: float = 12.0) -> dict:
     """The oracle as it stands, on whole sequences of the workload (all
-    heads), on this host's cores; tokens/s scaled from the sample."""
+    heads), on this host's cores; tokens/s scaled from the sample.  One
+    sequence is also run on a single thread."""
     import oracle
     threads = len(os.sched_getaffinity(0))
     lengths = [int(x) for x in inp["lengths"]]
@@ -242,10 +253,21 @@ def cpu_baseline_prefill(case, inp, max_seconds: float = 12.0) -> dict:
         tokens += n
         if t_total * (done + 1) / done > max_seconds:
             break
+    # the first sequence again on one thread (its first 1024 tokens at most)
+    n1 = min(1024, lengths[0])
+    sl1 = (slice(0, 1), slice(0, n1))
+    st1 = inp["state_in"][0:1] if inp["state_in"] is not None else None
+    t0 = time.perf_counter()
+    oracle.recurrence(inp["q"][sl1], inp["k"][sl1], inp["v"][sl1], inp["g"][sl1],
+                      inp["beta"][sl1], st1, oracle.dense_cu_seqlens(1, n1),
+                      per_key_gate=case.gate == "per_key", qdq=case.qdq, n_threads=1)
+    t1 = time.perf_counter() - t0
     return {"value": tokens / t_total, "unit": "tokens/s", "cores": threads, "kind": "oracle",
             "sample": f"{done} of {len(lengths)} sequences ({tokens} tokens x {case.H} heads), "
                       f"fp64 token recurrence + fp32 {case.qdq} codec, OpenMP over heads",
-            "seconds": round(t_total, 3)}
+            "seconds": round(t_total, 3), "value_1_thread": round(n1 / t1, 1),
+            "sample_1_thread": f"{n1} tokens x {case.H} heads of sequence 0",
+            "cpu_model": cpu_model()}
 
 
 def cpu_baseline_decode(case, inp, state) -> dict:
