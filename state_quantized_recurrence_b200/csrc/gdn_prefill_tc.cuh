@@ -277,9 +277,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   sm100::tc_fence_before();
   __syncthreads();
 
-  // Outputs of a chunk are computed in its last epilogue but stored at the
-  // start of the next chunk (or after the loop), off the state path: 32
-  // tokens x this thread's value row, packed as bf16 pairs.
+  // Outputs of a partial chunk (only a sequence's last can be one) are
+  // computed in its last epilogue and stored after the loop, directly: 32
+  // tokens x this thread's value row, packed as bf16 pairs.  Whole chunks
+  // leave through the output tile and TMA stores instead.
   uint32_t opk[16];
   __nv_bfloat16 *op_dst = nullptr;  // token 0 of the pending block, or null
   int op_cnt = 0;                   // valid tokens in it
@@ -340,7 +341,6 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       __syncwarp();
     }
 
-    flush_outputs();  // the previous chunk's outputs, while MMA 2 runs
 
     // ---- epilogue 1 (all warps; warps w and w + 4 split D1's 64 columns):
     //      rows 0-63 -> A (fp32, for the solve), rows 64-127 -> Aqk (fp16) ----
