@@ -18,7 +18,8 @@
  *     zero guard (PR #2497 What section); or dynamic INT8 with groups of 32
  *     along the last axis, scale = amax / 127, round half to even, clamp to
  *     [-127, 127] (PR #2519 commit notes, recipe
- *     linear_attention_state_int8_block32_dynamic);
+ *     linear_attention_state_int8_block32_dynamic); groups of 16 and 64 are
+ *     offered as well;
  *   - fp32 working values for the state and the gates, bf16 or fp32 q/k/v
  *     promoted to fp32 (PR #2519 commit notes).
  *
@@ -31,9 +32,11 @@
  *          GDN (GDN_GATE_SCALAR) or [.., H, d_k] for KDA (GDN_GATE_PER_KEY);
  *   beta   fp32 [.., H].
  *
- * Ownership: every pointer is caller-owned memory; the library allocates
- * nothing and keeps no reference after a call returns.  Pointers are device
- * pointers unless a function says otherwise.
+ * Ownership: every pointer is caller-owned memory; no call allocates memory
+ * and none keeps a reference after it returns.  The library's own device
+ * memory is a per-device error word and the 64 MiB scratch array of
+ * gdn_prefill_backward_static, both reserved when its module is loaded.
+ * Pointers are device pointers unless a function says otherwise.
  *
  * Asynchrony and errors: argument errors are detected on the host and
  * returned before anything is launched (nothing is written).  Compute calls
