@@ -64,6 +64,26 @@ __device__ __forceinline__ void store4(__nv_bfloat16 *p, float a, float b, float
 // together with x, by 2^64; power-of-two scaling is exact in both and keeps
 // 1/s finite, so the quotient is unchanged.  Quotients small enough to be
 // subnormal round to code 0 either way.
+// Packed fp32 pairs (sm_100 f32x2 arithmetic: each lane rounds exactly as
+// the scalar instruction, two lanes per instruction).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+  return d;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float &lo, float &hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
 struct ScaleRecip {
   float s;    // the scale itself (dequantization multiplies by it)
   float pre;  // exact power-of-two pre-scale of x and s (1 or 2^64)
@@ -85,6 +105,16 @@ __device__ __forceinline__ float div_by_scale(float x, const ScaleRecip &sr) {
   const float q0 = __fmul_rn(xs, sr.r);
   const float r = __fmaf_rn(-q0, sr.s2, xs);
   return __fmaf_rn(r, sr.r, q0);
+}
+
+// div_by_scale of two values in packed f32x2 arithmetic (the same roundings).
+__device__ __forceinline__ void div_by_scale2(float x0, float x1, const ScaleRecip &sr, float &q0,
+                                              float &q1) {
+  const uint64_t xs = f2_mul(f2_pack(x0, x1), f2_pack(sr.pre, sr.pre));
+  const uint64_t rr = f2_pack(sr.r, sr.r);
+  const uint64_t q = f2_mul(xs, rr);
+  const uint64_t res = f2_fma(q, f2_pack(-sr.s2, -sr.s2), xs);
+  f2_unpack(f2_fma(res, rr, q), q0, q1);
 }
 
 // INT8: c = clamp(rint(x / s), -127, 127); y = c * s.  s > 0.
@@ -111,6 +141,24 @@ __device__ __forceinline__ float2 qdq_fp8_2(float x0, float x1, const ScaleRecip
 
 // The codes themselves (for packed state storage); the dequantized values
 // of the functions above are exactly code * s.
+// INT8 codes and QDQ values of four values (two packed quotients).
+__device__ __forceinline__ float4 int8_code4(float4 x, const ScaleRecip &sr) {
+  float4 q;
+  div_by_scale2(x.x, x.y, sr, q.x, q.y);
+  div_by_scale2(x.z, x.w, sr, q.z, q.w);
+  return make_float4(fminf(fmaxf(rintf(q.x), -127.0f), 127.0f),
+                     fminf(fmaxf(rintf(q.y), -127.0f), 127.0f),
+                     fminf(fmaxf(rintf(q.z), -127.0f), 127.0f),
+                     fminf(fmaxf(rintf(q.w), -127.0f), 127.0f));
+}
+__device__ __forceinline__ float4 mul4(float4 c, float s) {
+  const uint64_t s2 = f2_pack(s, s);
+  float4 y;
+  f2_unpack(f2_mul(f2_pack(c.x, c.y), s2), y.x, y.y);
+  f2_unpack(f2_mul(f2_pack(c.z, c.w), s2), y.z, y.w);
+  return y;
+}
+
 __device__ __forceinline__ float int8_code(float x, const ScaleRecip &sr) {
   return fminf(fmaxf(rintf(div_by_scale(x, sr)), -127.0f), 127.0f);
 }

@@ -64,10 +64,9 @@ struct StateIO {
 #pragma unroll
         for (int j = 0; j < RPT; ++j) {
           const uint32_t w = cw[j];
-          h[j] = make_float4(__fmul_rn((float)(int8_t)(w & 0xffu), s[j]),
-                             __fmul_rn((float)(int8_t)((w >> 8) & 0xffu), s[j]),
-                             __fmul_rn((float)(int8_t)((w >> 16) & 0xffu), s[j]),
-                             __fmul_rn((float)(int8_t)(w >> 24), s[j]));
+          h[j] = mul4(make_float4((float)(int8_t)(w & 0xffu), (float)(int8_t)((w >> 8) & 0xffu),
+                                  (float)(int8_t)((w >> 16) & 0xffu), (float)(int8_t)(w >> 24)),
+                      s[j]);
         }
       } else {
         const float st = __ldg(sr.scales + col / 64);
@@ -99,14 +98,12 @@ struct StateIO {
         } else {
           const ScaleRecip s = make_scale(int8_scale(m));
           sc = s.s;
+          const float4 c = int8_code4(h[j], s);
           if (PACKED) {
-            const float c0 = int8_code(h[j].x, s), c1 = int8_code(h[j].y, s),
-                        c2 = int8_code(h[j].z, s), c3 = int8_code(h[j].w, s);
-            cw[j] = ((uint32_t)(uint8_t)(int8_t)c0) | ((uint32_t)(uint8_t)(int8_t)c1 << 8) |
-                    ((uint32_t)(uint8_t)(int8_t)c2 << 16) | ((uint32_t)(uint8_t)(int8_t)c3 << 24);
+            cw[j] = ((uint32_t)(uint8_t)(int8_t)c.x) | ((uint32_t)(uint8_t)(int8_t)c.y << 8) |
+                    ((uint32_t)(uint8_t)(int8_t)c.z << 16) | ((uint32_t)(uint8_t)(int8_t)c.w << 24);
           } else {
-            h[j].x = qdq_int8(h[j].x, s); h[j].y = qdq_int8(h[j].y, s);
-            h[j].z = qdq_int8(h[j].z, s); h[j].w = qdq_int8(h[j].w, s);
+            h[j] = mul4(c, s.s);
           }
         }
         if (PACKED && (col % GROUP) == 0)
@@ -178,15 +175,24 @@ __device__ __forceinline__ void decode_slab(float4 (&h)[DK / 16], const float *s
   kq = warp_sum(kq);
 
   // Decay and the partial key-axis reductions a = Ht^T k, b = Ht^T q.
-  float pa[4] = {0.f, 0.f, 0.f, 0.f}, pb[4] = {0.f, 0.f, 0.f, 0.f};
+  // (fp32 pairs in packed f32x2 arithmetic: each lane rounds as the scalar
+  // instruction)
+  uint64_t pa01 = 0, pa23 = 0, pb01 = 0, pb23 = 0;  // +0.0 pairs
 #pragma unroll
   for (int j = 0; j < RPT; ++j) {
     const int r = rg + 16 * j;
     const float al = PER_KEY ? s_al[r] : a_scalar, kr = s_k[r], qr = s_q[r];
-    h[j].x *= al; h[j].y *= al; h[j].z *= al; h[j].w *= al;
-    pa[0] += h[j].x * kr; pa[1] += h[j].y * kr; pa[2] += h[j].z * kr; pa[3] += h[j].w * kr;
-    pb[0] += h[j].x * qr; pb[1] += h[j].y * qr; pb[2] += h[j].z * qr; pb[3] += h[j].w * qr;
+    const uint64_t al2 = f2_pack(al, al), kr2 = f2_pack(kr, kr), qr2 = f2_pack(qr, qr);
+    const uint64_t h01 = f2_mul(f2_pack(h[j].x, h[j].y), al2);
+    const uint64_t h23 = f2_mul(f2_pack(h[j].z, h[j].w), al2);
+    f2_unpack(h01, h[j].x, h[j].y);
+    f2_unpack(h23, h[j].z, h[j].w);
+    pa01 = f2_fma(h01, kr2, pa01); pa23 = f2_fma(h23, kr2, pa23);
+    pb01 = f2_fma(h01, qr2, pb01); pb23 = f2_fma(h23, qr2, pb23);
   }
+  float pa[4], pb[4];
+  f2_unpack(pa01, pa[0], pa[1]); f2_unpack(pa23, pa[2], pa[3]);
+  f2_unpack(pb01, pb[0], pb[1]); f2_unpack(pb23, pb[2], pb[3]);
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
     pa[e] += __shfl_xor_sync(0xffffffffu, pa[e], 16);
@@ -212,11 +218,13 @@ __device__ __forceinline__ void decode_slab(float4 (&h)[DK / 16], const float *s
            scale * fmaf(kq, u[2], b[2]), scale * fmaf(kq, u[3], b[3]));
 
   // Delta update H = Ht + k u^T.
+  const uint64_t u01 = f2_pack(u[0], u[1]), u23 = f2_pack(u[2], u[3]);
 #pragma unroll
   for (int j = 0; j < RPT; ++j) {
     const float kr = s_k[rg + 16 * j];
-    h[j].x = fmaf(kr, u[0], h[j].x); h[j].y = fmaf(kr, u[1], h[j].y);
-    h[j].z = fmaf(kr, u[2], h[j].z); h[j].w = fmaf(kr, u[3], h[j].w);
+    const uint64_t kr2 = f2_pack(kr, kr);
+    f2_unpack(f2_fma(kr2, u01, f2_pack(h[j].x, h[j].y)), h[j].x, h[j].y);
+    f2_unpack(f2_fma(kr2, u23, f2_pack(h[j].z, h[j].w)), h[j].z, h[j].w);
   }
 
   // State QDQ and store.

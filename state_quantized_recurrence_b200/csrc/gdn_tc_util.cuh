@@ -63,26 +63,6 @@ __device__ __forceinline__ void store32_hl(uint32_t thi, uint32_t tlo, int r, in
   }
 }
 
-// Packed fp32 pairs (sm_100 f32x2 arithmetic: each lane rounds exactly as
-// the scalar instruction, two lanes per instruction).
-__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
-  uint64_t d;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
-  return d;
-}
-__device__ __forceinline__ void f2_unpack(uint64_t v, float &lo, float &hi) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
 // y[i] *= s for 32 values.
 __device__ __forceinline__ void scale32(float *y, float s) {
   const uint64_t s2 = f2_pack(s, s);
