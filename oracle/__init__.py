@@ -17,7 +17,9 @@ Modes:
 
 Pins: every function here is checked by ``tests/test_oracle_*.py`` against
 closed forms, invariants, special cases and library routines (see the
-tests' docstrings).  Nothing stored or computed here comes from the CUDA path.
+tests' docstrings); ``tests/test_oracle_mutants.py`` plants single mistakes
+in copies of the C recurrence, the codecs and the chunked form and requires
+each to fail a pin.  Nothing stored or computed here comes from the CUDA path.
 """
 
 from __future__ import annotations
@@ -42,17 +44,18 @@ _QDQ_GROUP = {"int8_g32": 32, "int8_g16": 16, "int8_g64": 64}
 CHUNK = 64
 
 
-def build(force: bool = False) -> str:
-    """Compile ``liboracle.so`` with gcc (no fast-math, no FP contraction)."""
-    if (not force and os.path.exists(_LIB)
-            and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC)):
-        return _LIB
+def build(force: bool = False, src: str = _SRC, out: str = _LIB) -> str:
+    """Compile ``liboracle.so`` with gcc (no fast-math, no FP contraction).
+    ``src``/``out`` let the tests compile a copy with a planted mistake."""
+    if (not force and os.path.exists(out)
+            and os.path.getmtime(out) >= os.path.getmtime(src)):
+        return out
     cmd = ["gcc", "-std=c11", "-O2", "-fPIC", "-shared", "-fopenmp",
            "-fno-fast-math", "-ffp-contract=off", "-fno-finite-math-only",
-           "-o", _LIB + ".tmp", _SRC, "-lm"]
+           "-o", out + ".tmp", src, "-lm"]
     subprocess.run(cmd, check=True)
-    os.replace(_LIB + ".tmp", _LIB)
-    return _LIB
+    os.replace(out + ".tmp", out)
+    return out
 
 
 _lib = None
@@ -61,22 +64,26 @@ _lib = None
 def _load():
     global _lib
     if _lib is None:
-        build()
-        lib = ctypes.CDLL(_LIB)
-        P = ctypes.c_void_p
-        lib.or_e4m3_rne_satfinite.argtypes = [ctypes.c_float]
-        lib.or_e4m3_rne_satfinite.restype = ctypes.c_float
-        lib.or_e4m3_array.argtypes = [P, P, ctypes.c_long]
-        lib.or_e4m3_array.restype = None
-        lib.or_qdq.argtypes = [P, ctypes.c_long, ctypes.c_int, ctypes.c_int,
-                               ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P]
-        lib.or_qdq.restype = ctypes.c_int
-        lib.or_gdn_recurrence.argtypes = [P] * 7 + [ctypes.c_int] * 9 + [P] * 4 + [ctypes.c_int]
-        lib.or_gdn_recurrence.restype = ctypes.c_int
-        lib.or_max_threads.argtypes = []
-        lib.or_max_threads.restype = ctypes.c_int
-        _lib = lib
+        _lib = bind(build())
     return _lib
+
+
+def bind(path: str):
+    """Load a compiled oracle library and declare its entry points."""
+    lib = ctypes.CDLL(path)
+    P = ctypes.c_void_p
+    lib.or_e4m3_rne_satfinite.argtypes = [ctypes.c_float]
+    lib.or_e4m3_rne_satfinite.restype = ctypes.c_float
+    lib.or_e4m3_array.argtypes = [P, P, ctypes.c_long]
+    lib.or_e4m3_array.restype = None
+    lib.or_qdq.argtypes = [P, ctypes.c_long, ctypes.c_int, ctypes.c_int,
+                           ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P]
+    lib.or_qdq.restype = ctypes.c_int
+    lib.or_gdn_recurrence.argtypes = [P] * 7 + [ctypes.c_int] * 9 + [P] * 4 + [ctypes.c_int]
+    lib.or_gdn_recurrence.restype = ctypes.c_int
+    lib.or_max_threads.argtypes = []
+    lib.or_max_threads.restype = ctypes.c_int
+    return lib
 
 
 def _ptr(a: Optional[np.ndarray]):
