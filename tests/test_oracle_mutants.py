@@ -10,9 +10,9 @@ copy, and requires that some pin fails.
 * C token recurrence and codecs: a copy of ``gdn_oracle.c`` with one textual
   change is compiled with the oracle's own flags into a temporary library and
   swapped in for the duration of the case;
-* fp64 chunked WY form: a copy of ``oracle/chunked.py`` with one textual
-  change is loaded as a module and swapped in for the pin module's
-  reference to it.
+* fp64 chunked WY form and fp64 backward: a copy of ``oracle/chunked.py`` or
+  ``oracle/backward.py`` with one textual change is loaded as a module and
+  swapped in for the pin module's reference to it.
 
 The oracle itself is never modified on disk; every case restores it.
 """
@@ -23,6 +23,7 @@ import types
 import pytest
 
 import oracle
+import test_oracle_backward as bwd
 import test_oracle_codecs as codecs
 import test_oracle_recurrence as rec
 
@@ -91,6 +92,40 @@ PY_MUTANTS = [
     ("Neumann one term short", "for _ in range(degree):", "for _ in range(degree - 1):"),
 ]
 
+BWD_MUTANTS = [
+    ("dq without the scale", "dq[tok, h] = scale * (Hn @ do[tok, h])",
+     "dq[tok, h] = Hn @ do[tok, h]"),
+    ("dq from the pre-update state", "dq[tok, h] = scale * (Hn @ do[tok, h])",
+     "dq[tok, h] = scale * (Ht @ do[tok, h])"),
+    ("output adjoint dropped", "dHn = dH + scale * np.outer(qt, do[tok, h])", "dHn = dH"),
+    ("dbeta sign", "dbeta[tok, h] = du @ (vt - a)", "dbeta[tok, h] = du @ (vt + a)"),
+    ("dv without beta", "dv[tok, h] = bt * du", "dv[tok, h] = du"),
+    ("retrieval adjoint sign", "da = -bt * du", "da = bt * du"),
+    ("dk misses the retrieval path", "dkt = dkt + Ht @ da", "dkt = dkt"),
+    ("gate adjoint from the decayed state", "dal = np.sum(Hp * dHt, axis=1)",
+     "dal = np.sum(Ht * dHt, axis=1)"),
+    ("scalar gate adjoint without alpha", "dg[tok, h] = al[0] * dal.sum()",
+     "dg[tok, h] = dal.sum()"),
+    ("state adjoint not decayed", "dH = al[:, None] * dHt", "dH = dHt"),
+    ("reverse pass off the quantized trajectory",
+     "per_key_gate=per_key_gate, qdq=qdq,\n                              boundary_every=boundary_every, record=True)",
+     "per_key_gate=per_key_gate, qdq=\"none\",\n                              boundary_every=boundary_every, record=True)"),
+    ("forward misses the partial last chunk", "return (t + 1) % every == 0 or t == L - 1",
+     "return (t + 1) % every == 0"),
+]
+
+BWD_PINS = [
+    ("closed forms", bwd.test_backward_closed_forms_constant_state),
+    ("python forward = C (gdn, int8)",
+     lambda: bwd.test_python_forward_matches_c_recurrence(False, "int8_g32")),
+    ("python forward = C (kda, fp8)",
+     lambda: bwd.test_python_forward_matches_c_recurrence(True, "fp8_tile64")),
+    ("finite differences (gdn)", lambda: bwd.test_backward_matches_finite_differences_qdq_off(False)),
+    ("finite differences (kda)", lambda: bwd.test_backward_matches_finite_differences_qdq_off(True)),
+    ("straight through (gdn, fp8)", lambda: bwd.test_backward_is_straight_through(False, "fp8_tile64")),
+    ("straight through (kda, int8)", lambda: bwd.test_backward_is_straight_through(True, "int8_g32")),
+]
+
 # The pins, cheapest first: a case stops at the first one that fails.
 PINS = [
     ("golden fp8 tile", codecs.test_golden_fp8_tile),
@@ -123,8 +158,8 @@ PINS = [
 ]
 
 
-def first_failing_pin():
-    for name, pin in PINS:
+def first_failing_pin(pins=None):
+    for name, pin in PINS if pins is None else pins:
         try:
             pin()
         except Exception:  # an assertion, or arithmetic the mistake broke
@@ -139,6 +174,7 @@ def _plant(text, old, new, what):
 
 def test_pins_pass_on_the_oracle_itself():
     assert first_failing_pin() is None
+    assert first_failing_pin(BWD_PINS) is None
 
 
 @pytest.mark.parametrize("name,old,new", C_MUTANTS, ids=[m[0] for m in C_MUTANTS])
@@ -161,3 +197,15 @@ def test_planted_chunked_mistake_fails_a_pin(name, old, new, monkeypatch):
     exec(compile(src, path + " (mutant)", "exec"), mod.__dict__)
     monkeypatch.setattr(rec, "chunked", mod)
     assert first_failing_pin() is not None, f"no pin fails with the mistake '{name}'"
+
+
+@pytest.mark.parametrize("name,old,new", BWD_MUTANTS, ids=[m[0] for m in BWD_MUTANTS])
+def test_planted_backward_mistake_fails_a_pin(name, old, new, monkeypatch):
+    path = os.path.join(os.path.dirname(oracle.__file__), "backward.py")
+    src = _plant(open(path).read(), old, new, name)
+    mod = types.ModuleType("oracle.backward_mutant")
+    mod.__package__ = "oracle"
+    mod.__file__ = path
+    exec(compile(src, path + " (mutant)", "exec"), mod.__dict__)
+    monkeypatch.setattr(bwd, "bw", mod)
+    assert first_failing_pin(BWD_PINS) is not None, f"no pin fails with the mistake '{name}'"
