@@ -19,8 +19,7 @@ Pins: every function here is checked by ``tests/test_oracle_*.py`` against
 closed forms, invariants, special cases and library routines (see the
 tests' docstrings); ``tests/test_oracle_mutants.py`` plants single mistakes
 in copies of the C recurrence, the codecs, the chunked form and the backward
-and requires
-each to fail a pin.  Nothing stored or computed here comes from the CUDA path.
+and requires each to fail a pin.  Nothing stored or computed here comes from the CUDA path.
 """
 
 from __future__ import annotations
