@@ -108,7 +108,10 @@ typedef enum {
  * triangular solve a chunk ahead, the other carries the state).  Pairs are
  * used when every (sequence, head) gets its pair in one wave on the current
  * device; the environment variable GDN_PREFILL_CTA_PAIR=0 or =1, read at
- * every call, forces one CTA or the pair.
+ * every call, forces one CTA or the pair.  Every other combination (fp32
+ * q/k/v, KDA gates, d_k or d_v = 64) runs a CUDA-core kernel with one CTA
+ * per (sequence, head, 64-column value tile) computing the same chunked
+ * form in fp32.  gdn_prefill_schedule() reports which kernel a shape gets.
  *
  * Returns GDN_OK after a successful launch (or when there is no work).
  */
