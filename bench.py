@@ -660,7 +660,7 @@ def run_decode(args, dist, dev, stream, sampler, peaks, packed: bool = False) ->
 # ------------------------------------------------------------ reference arm
 def run_reference(args, dist: Dist) -> dict | None:
     """The oracle, as it stands, on the host cores: each step is a bounded
-    sample (one sequence, all heads, the first 1024 tokens) of the workload."""
+    sample (the first sequence, all heads, all 4096 tokens) of the workload."""
     if dist.rank != 0:
         return None
     import gdn_synth as gs
