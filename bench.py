@@ -9,7 +9,14 @@ q/k/v, fp32 gates/state, FP8 E4M3 tile-64 state QDQ at every 64-token
 chunk): one step = one gdn_prefill call over the whole batch with inputs
 resident in HBM.  The serving-decode workload (256 sequences x 32 heads,
 d=128, INT8 g32 state QDQ after every token, 512 single-token gdn_decode
-calls) is measured in the same run and reported under "decode".
+calls) is measured in the same run and reported under "decode", the same
+with the state stored packed under "decode_packed", one straight-through
+backward call on the GDN-prefill workload under "backward", and the KDA and
+packed-varlen prefill workloads under "prefill_other".  Beside each:
+`roofline` (algorithmic bytes or flops per launch over the CUDA-event time,
+against the measured peaks, with the DRAM traffic recorded by ncu for the
+same sources), `cpu_baseline` (the oracle on the host cores) and, for the
+headline, `e2e` (the same call with pinned host copies in the timed region).
 
 With N > 1 (torchrun, one rank per GPU) every rank runs its own copy of the
 workload (independent sequences; no collective on the data path), the step
