@@ -8,6 +8,8 @@ library is missing.
 
     o, state = gdn_prefill(q, k, v, g, beta, state_in=None, cu_seqlens=None,
                            qdq="fp8_tile64")
+    o, state = gdn_prefill(..., neumann_degree=7)   # approximate solve, 2^m - 1
+    gdn_prefill_schedule(n_seq, H, d_k, d_v)        # which prefill kernel runs
     o = gdn_decode(q, k, v, g, beta, state, qdq="int8_g32")   # state in place
     dq, dk, dv, dg, dbeta, dstate_in = gdn_prefill_backward(q, k, v, g, beta, d_o, ...)
 

@@ -249,7 +249,10 @@ def gdn_prefill_backward_static(q, k, v, g, beta, d_o, state_in=None, cu_seqlens
 
 def gdn_prefill(q, k, v, g, beta, state_in=None, cu_seqlens=None, qdq: str = "fp8_tile64",
                 stream=None, neumann_degree: Optional[int] = None):
-    """Chunked prefix; returns ``(o, state_out)`` (allocated with torch)."""
+    """Chunked prefix; returns ``(o, state_out)`` (allocated with torch).
+    ``neumann_degree`` (1, 3, 7, 15, 31 or 63) replaces the exact triangular
+    solve of every chunk by the truncated Neumann series of that degree
+    (``gdn_prefill_neumann``); None keeps the exact solve (``gdn_prefill``)."""
     n_seq = q.shape[0] if cu_seqlens is None else cu_seqlens.numel() - 1
     o = torch.empty(v.shape, dtype=q.dtype, device=q.device)
     state_out = torch.empty((n_seq, q.shape[2], q.shape[3], v.shape[3]), dtype=torch.float32,
