@@ -416,10 +416,12 @@ def measure_prefill(args, dist, dev, stream, sampler, peaks, case, steps, warmup
     flops = prefill_flops(tokens, case.H, case.d_k, case.d_v)
     gbs = nbytes / (ms / 1e3) / 1e9
     tfs = flops / (ms / 1e3) / 1e12
-    kernel = {"tc_cta_pair": "pair::prefill_pair_kernel (tcgen05, CTA pair per unit)",
+    kernel = {"tc_wy_pair": "wy::prefill_wy_kernel (tcgen05, WY-form CTA pair per unit)",
+              "tc_cta_pair": "pair::prefill_pair_kernel (tcgen05, CTA pair per unit)",
               "tc_one_cta": "tc::prefill_tc_kernel (tcgen05, one CTA per unit)",
               "cuda_cores": "simt::prefill_simt_kernel (FFMA)"}[
-        sqr.gdn_prefill_schedule(case.n_seq, case.H, case.d_k, case.d_v, d["q"].dtype, case.gate)]
+        sqr.gdn_prefill_schedule(case.n_seq, case.H, case.d_k, case.d_v, d["q"].dtype, case.gate,
+                                 case.qdq)]
     res = {
         "workload": f"{case.name}: n_seq={case.n_seq} H={case.H} tokens={tokens} d={case.d_k}, "
                     f"{case.dtype}, {case.gate} gate, {case.qdq}, "
@@ -521,6 +523,29 @@ def run_ours(args, dist: Dist) -> dict:
                                3, 3)
 
     sampler.stop()
+
+    def pick(d, *path):
+        for k in path:
+            if not isinstance(d, dict) or d.get(k) is None:
+                return None
+            d = d[k]
+        return d
+
+    # the other targets, flat at the top level of the line
+    flat = {
+        "tensor_frac": pick(roofline, "tensor", "frac"),
+        "decode_updates_per_s": pick(dec, "value"),
+        "decode_ms_per_token_step": pick(dec, "ms_per_token_step"),
+        "decode_hbm_frac": pick(dec, "roofline", "frac"),
+        "decode_packed_updates_per_s": pick(dec_packed, "value"),
+        "decode_packed_hbm_frac": pick(dec_packed, "roofline", "frac"),
+        "kda_ms_per_step": pick(others, "kda_prefill", "ms_per_step"),
+        "kda_hbm_frac": pick(others, "kda_prefill", "roofline", "frac"),
+        "varlen_ms_per_step": pick(others, "varlen", "ms_per_step"),
+        "varlen_hbm_frac": pick(others, "varlen", "roofline", "frac"),
+        "backward_ms_per_step": pick(bwd, "ms_per_step"),
+        "backward_hbm_frac": pick(bwd, "roofline", "frac"),
+    }
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": dist.world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_max, 5),
@@ -534,6 +559,7 @@ def run_ours(args, dist: Dist) -> dict:
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps,
         "clocks": clocks, "decode": dec, "decode_packed": dec_packed,
         "prefill_other": others or None, "backward": bwd, "impl": "ours",
+        **flat,
     }
     dist.close()
     return res

@@ -267,19 +267,21 @@ gdn_status gdn_prefill_backward_static(const void *q, const void *k, const void 
 
 /*
  * gdn_prefill_schedule - which prefill kernel gdn_prefill launches for these
- * shapes on the current device, under the current GDN_PREFILL_CTA_PAIR
- * setting (the same selection code).  Host-only; it may query the device's
- * cluster occupancy once.  Returns a gdn_prefill_kernel value, or -1 for
- * arguments gdn_prefill would reject as invalid or unsupported.  This has no
- * counterpart in the method's description: it reports an implementation
- * choice.
+ * shapes and this codec on the current device, under the current
+ * GDN_PREFILL_CTA_PAIR and GDN_PREFILL_WY settings (the same selection code).
+ * Host-only; it may query the device's cluster occupancy once.  Returns a
+ * gdn_prefill_kernel value, or -1 for arguments gdn_prefill would reject as
+ * invalid or unsupported.  This has no counterpart in the method's
+ * description: it reports an implementation choice.
  */
 typedef enum {
     GDN_PREFILL_CUDA_CORES = 0,   /* fp32, KDA or d = 64: FFMA kernel */
     GDN_PREFILL_TC_ONE_CTA = 1,   /* tensor cores, one CTA per (sequence, head) */
-    GDN_PREFILL_TC_CTA_PAIR = 2   /* tensor cores, a CTA pair per (sequence, head) */
+    GDN_PREFILL_TC_CTA_PAIR = 2,  /* tensor cores, a CTA pair per (sequence, head) */
+    GDN_PREFILL_TC_WY_PAIR = 3    /* tensor cores, a CTA pair in the WY form (FP8 tiles) */
 } gdn_prefill_kernel;
-int gdn_prefill_schedule(int n_seq, int H, int d_k, int d_v, gdn_dtype dt, gdn_gate_kind gk);
+int gdn_prefill_schedule(int n_seq, int H, int d_k, int d_v, gdn_dtype dt, gdn_gate_kind gk,
+                         gdn_qdq_mode qdq);
 
 /* gdn_status_string - static, human-readable name of a status code. */
 const char *gdn_status_string(gdn_status s);

@@ -56,7 +56,7 @@ def _load() -> ctypes.CDLL:
     L.gdn_status_string.restype = ctypes.c_char_p
     L.gdn_version.argtypes = []
     L.gdn_version.restype = I
-    L.gdn_prefill_schedule.argtypes = [I, I, I, I, I, I]
+    L.gdn_prefill_schedule.argtypes = [I, I, I, I, I, I, I]
     L.gdn_prefill_schedule.restype = I
     return L
 
@@ -68,9 +68,11 @@ def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _stream(stream) -> ctypes.c_void_p:
+def _stream(stream, device=None) -> ctypes.c_void_p:
+    """The given stream, else the current stream of ``device`` (default: the
+    current device)."""
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(device)
     return ctypes.c_void_p(stream.cuda_stream)
 
 
@@ -79,33 +81,48 @@ def _need(cond: bool, msg: str):
         raise ValueError(msg)
 
 
-def _check_dev(*ts):
+def _check_dev(*ts) -> torch.device:
+    """Every tensor a contiguous CUDA tensor on one device; returns it.  The
+    library launches on the current device, so each call below makes this
+    device current around the C call (and takes its current stream)."""
+    dev = None
     for t in ts:
         if t is not None:
             _need(t.is_cuda and t.is_contiguous(), "tensors must be contiguous CUDA tensors")
+            if dev is None:
+                dev = t.device
+            _need(t.device == dev, f"tensors on different devices ({dev} and {t.device})")
+    return dev
 
 
-GDN_PREFILL_KERNEL = {0: "cuda_cores", 1: "tc_one_cta", 2: "tc_cta_pair"}
+GDN_PREFILL_KERNEL = {0: "cuda_cores", 1: "tc_one_cta", 2: "tc_cta_pair", 3: "tc_wy_pair"}
 
 
 def gdn_prefill_schedule(n_seq: int, H: int, d_k: int, d_v: int, dtype=torch.bfloat16,
-                         gate: str = "scalar") -> str:
-    """Which prefill kernel gdn_prefill launches for these shapes on the
-    current device: "cuda_cores", "tc_one_cta" or "tc_cta_pair"."""
-    _need(dtype in GDN_DTYPE and gate in GDN_GATE, "unsupported dtype or gate kind")
+                         gate: str = "scalar", qdq: str = "fp8_tile64") -> str:
+    """Which prefill kernel gdn_prefill launches for these shapes and this
+    codec on the current device: "cuda_cores", "tc_one_cta", "tc_cta_pair"
+    or "tc_wy_pair"."""
+    _need(dtype in GDN_DTYPE and gate in GDN_GATE and qdq in GDN_QDQ,
+          "unsupported dtype, gate kind or codec")
     r = int(lib.gdn_prefill_schedule(int(n_seq), int(H), int(d_k), int(d_v), GDN_DTYPE[dtype],
-                                     GDN_GATE[gate]))
+                                     GDN_GATE[gate], GDN_QDQ[qdq]))
     _need(r >= 0, "shapes gdn_prefill does not support")
     return GDN_PREFILL_KERNEL[r]
 
 
-def gdn_last_error(stream=None) -> int:
-    """Synchronize the stream and return (and clear) the device error status."""
-    return int(lib.gdn_last_error(_stream(stream)))
+def gdn_last_error(stream=None, device=None) -> int:
+    """Synchronize the stream (default: the current stream of ``device``, or
+    of the current device) and return (and clear) that device's error
+    status."""
+    if device is None:
+        device = stream.device if stream is not None else torch.cuda.current_device()
+    with torch.cuda.device(device):
+        return int(lib.gdn_last_error(_stream(stream, device)))
 
 
-def check_last_error(stream=None, where: str = "gdn") -> None:
-    s = gdn_last_error(stream)
+def check_last_error(stream=None, where: str = "gdn", device=None) -> None:
+    s = gdn_last_error(stream, device)
     if s != 0:
         raise GdnError(s, where)
 
@@ -125,7 +142,7 @@ def gdn_prefill_into(q, k, v, g, beta, state_in, cu_seqlens, o, state_out,
     (1, 3, 7, 15, 31 or 63) selects the approximate solve
     (gdn_prefill_neumann); None the exact one.
     """
-    _check_dev(q, k, v, g, beta, state_in, cu_seqlens, o, state_out)
+    dev = _check_dev(q, k, v, g, beta, state_in, cu_seqlens, o, state_out)
     _need(q.dim() == 4 and k.shape == q.shape and v.dim() == 4, "q, k, v must be [B, T, H, d]")
     B, T, H, d_k = q.shape
     d_v = v.shape[-1]
@@ -149,11 +166,13 @@ def gdn_prefill_into(q, k, v, g, beta, state_in, cu_seqlens, o, state_out,
               "state_in must be fp32 [n_seq, H, d_k, d_v]")
     args = (_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_in), _ptr(cu_seqlens),
             n_seq, T_arg, H, d_k, d_v, GDN_DTYPE[q.dtype], GDN_GATE[gk], GDN_QDQ[qdq])
-    tail = (_ptr(o), _ptr(state_out), _stream(stream))
-    if neumann_degree is None:
-        s, where = lib.gdn_prefill(*args, *tail), "gdn_prefill"
-    else:
-        s, where = lib.gdn_prefill_neumann(*args, int(neumann_degree), *tail), "gdn_prefill_neumann"
+    with torch.cuda.device(dev):
+        tail = (_ptr(o), _ptr(state_out), _stream(stream, dev))
+        if neumann_degree is None:
+            s, where = lib.gdn_prefill(*args, *tail), "gdn_prefill"
+        else:
+            s, where = (lib.gdn_prefill_neumann(*args, int(neumann_degree), *tail),
+                        "gdn_prefill_neumann")
     if s != 0:
         raise GdnError(s, where)
 
@@ -167,7 +186,7 @@ def gdn_prefill_backward(q, k, v, g, beta, d_o, state_in=None, cu_seqlens=None,
     through.  Returns fp32 ``(dq, dk, dv, dg, dbeta, dstate_in)``.
     ``workspace``: a CUDA uint8 tensor of at least
     gdn_prefill_backward_workspace_bytes(...) bytes, or None to allocate one."""
-    _check_dev(q, k, v, g, beta, d_o, state_in, cu_seqlens, dstate_out, workspace)
+    dev = _check_dev(q, k, v, g, beta, d_o, state_in, cu_seqlens, dstate_out, workspace)
     _need(q.dim() == 4 and k.shape == q.shape and v.dim() == 4, "q, k, v must be [B, T, H, d]")
     B, T, H, d_k = q.shape
     d_v = v.shape[-1]
@@ -196,11 +215,12 @@ def gdn_prefill_backward(q, k, v, g, beta, d_o, state_in=None, cu_seqlens=None,
     dv = torch.empty(v.shape, **f32)
     dg, dbeta = torch.empty(g.shape, **f32), torch.empty(beta.shape, **f32)
     dstate_in = torch.empty(sshape, **f32)
-    s = lib.gdn_prefill_backward(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_in), _ptr(cu_seqlens), n_seq,
-        T_arg, H, d_k, d_v, GDN_DTYPE[q.dtype], GDN_GATE[gk], GDN_QDQ[qdq], _ptr(d_o),
-        _ptr(dstate_out), _ptr(workspace), workspace.numel(), _ptr(dq), _ptr(dk), _ptr(dv),
-        _ptr(dg), _ptr(dbeta), _ptr(dstate_in), _stream(stream))
+    with torch.cuda.device(dev):
+        s = lib.gdn_prefill_backward(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_in), _ptr(cu_seqlens), n_seq,
+            T_arg, H, d_k, d_v, GDN_DTYPE[q.dtype], GDN_GATE[gk], GDN_QDQ[qdq], _ptr(d_o),
+            _ptr(dstate_out), _ptr(workspace), workspace.numel(), _ptr(dq), _ptr(dk), _ptr(dv),
+            _ptr(dg), _ptr(dbeta), _ptr(dstate_in), _stream(stream, dev))
     if s != 0:
         raise GdnError(s, "gdn_prefill_backward")
     return dq, dk, dv, dg, dbeta, dstate_in
@@ -212,7 +232,7 @@ def gdn_prefill_backward_static(q, k, v, g, beta, d_o, state_in=None, cu_seqlens
     static device array (64 MiB; larger problems raise GDN_ERR_UNSUPPORTED).
     Calls that overlap on one device share that array: order them.  Returns
     fp32 ``(dq, dk, dv, dg, dbeta, dstate_in)`` (allocated here with torch)."""
-    _check_dev(q, k, v, g, beta, d_o, state_in, cu_seqlens, dstate_out)
+    dev = _check_dev(q, k, v, g, beta, d_o, state_in, cu_seqlens, dstate_out)
     _need(q.dim() == 4 and k.shape == q.shape and v.dim() == 4, "q, k, v must be [B, T, H, d]")
     B, T, H, d_k = q.shape
     d_v = v.shape[-1]
@@ -237,11 +257,12 @@ def gdn_prefill_backward_static(q, k, v, g, beta, d_o, state_in=None, cu_seqlens
     dv = torch.empty(v.shape, **f32)
     dg, dbeta = torch.empty(g.shape, **f32), torch.empty(beta.shape, **f32)
     dstate_in = torch.empty(sshape, **f32)
-    s = lib.gdn_prefill_backward_static(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_in), _ptr(cu_seqlens), n_seq,
-        T_arg, H, d_k, d_v, GDN_DTYPE[q.dtype], GDN_GATE[gk], GDN_QDQ[qdq], _ptr(d_o),
-        _ptr(dstate_out), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg), _ptr(dbeta), _ptr(dstate_in),
-        _stream(stream))
+    with torch.cuda.device(dev):
+        s = lib.gdn_prefill_backward_static(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_in), _ptr(cu_seqlens), n_seq,
+            T_arg, H, d_k, d_v, GDN_DTYPE[q.dtype], GDN_GATE[gk], GDN_QDQ[qdq], _ptr(d_o),
+            _ptr(dstate_out), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg), _ptr(dbeta), _ptr(dstate_in),
+            _stream(stream, dev))
     if s != 0:
         raise GdnError(s, "gdn_prefill_backward_static")
     return dq, dk, dv, dg, dbeta, dstate_in
@@ -266,7 +287,7 @@ def gdn_decode_into(q, k, v, g, beta, state, o, qdq: str = "int8_g32", stream=No
     """One decode token per sequence: q, k [N, H, d_k], v/o [N, H, d_v],
     g [N, H] or [N, H, d_k], beta [N, H]; ``state`` [N, H, d_k, d_v] fp32 is
     advanced and QDQ'd in place."""
-    _check_dev(q, k, v, g, beta, state, o)
+    dev = _check_dev(q, k, v, g, beta, state, o)
     _need(q.dim() == 3 and k.shape == q.shape and v.dim() == 3 and o.shape == v.shape,
           "q, k [N, H, d_k]; v, o [N, H, d_v]")
     N, H, d_k = q.shape
@@ -279,9 +300,10 @@ def gdn_decode_into(q, k, v, g, beta, state, o, qdq: str = "int8_g32", stream=No
     _need(g.shape == ((N, H) if gk == "scalar" else (N, H, d_k)), "g must be [N,H] or [N,H,d_k]")
     _need(state.shape == (N, H, d_k, d_v) and state.dtype == torch.float32,
           "state must be fp32 [N, H, d_k, d_v]")
-    s = lib.gdn_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state), N, H, d_k,
-                       d_v, GDN_DTYPE[q.dtype], GDN_GATE[gk], GDN_QDQ[qdq], _ptr(o),
-                       _stream(stream))
+    with torch.cuda.device(dev):
+        s = lib.gdn_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state), N, H, d_k,
+                           d_v, GDN_DTYPE[q.dtype], GDN_GATE[gk], GDN_QDQ[qdq], _ptr(o),
+                           _stream(stream, dev))
     if s != 0:
         raise GdnError(s, "gdn_decode")
 
@@ -325,10 +347,11 @@ def gdn_state_pack(state: torch.Tensor, qdq: str, out: Optional[PackedState] = N
     _need(state.dim() == 4 and state.dtype == torch.float32, "state must be fp32 [N, H, d_k, d_v]")
     N, H, d_k, d_v = state.shape
     ps = out if out is not None else packed_state_empty(N, H, d_k, d_v, qdq, state.device)
-    _check_dev(state, ps.codes, ps.scales)
+    dev = _check_dev(state, ps.codes, ps.scales)
     _need(ps.shape == tuple(state.shape) and ps.qdq == qdq, "packed state shape / mode mismatch")
-    s = lib.gdn_state_pack(_ptr(state), _ptr(ps.codes), _ptr(ps.scales), N, H, d_k, d_v,
-                           GDN_QDQ[qdq], _stream(stream))
+    with torch.cuda.device(dev):
+        s = lib.gdn_state_pack(_ptr(state), _ptr(ps.codes), _ptr(ps.scales), N, H, d_k, d_v,
+                               GDN_QDQ[qdq], _stream(stream, dev))
     if s != 0:
         raise GdnError(s, "gdn_state_pack")
     return ps
@@ -339,9 +362,10 @@ def gdn_state_unpack(ps: PackedState, out: Optional[torch.Tensor] = None, stream
     N, H, d_k, d_v = ps.shape
     st = out if out is not None else torch.empty((N, H, d_k, d_v), dtype=torch.float32,
                                                  device=ps.codes.device)
-    _check_dev(st, ps.codes, ps.scales)
-    s = lib.gdn_state_unpack(_ptr(ps.codes), _ptr(ps.scales), _ptr(st), N, H, d_k, d_v,
-                             GDN_QDQ[ps.qdq], _stream(stream))
+    dev = _check_dev(st, ps.codes, ps.scales)
+    with torch.cuda.device(dev):
+        s = lib.gdn_state_unpack(_ptr(ps.codes), _ptr(ps.scales), _ptr(st), N, H, d_k, d_v,
+                                 GDN_QDQ[ps.qdq], _stream(stream, dev))
     if s != 0:
         raise GdnError(s, "gdn_state_unpack")
     return st
@@ -349,7 +373,7 @@ def gdn_state_unpack(ps: PackedState, out: Optional[torch.Tensor] = None, stream
 
 def gdn_decode_packed_into(q, k, v, g, beta, ps: PackedState, o, stream=None) -> None:
     """gdn_decode_into with the state stored packed (updated in place)."""
-    _check_dev(q, k, v, g, beta, ps.codes, ps.scales, o)
+    dev = _check_dev(q, k, v, g, beta, ps.codes, ps.scales, o)
     _need(q.dim() == 3 and k.shape == q.shape and v.dim() == 3 and o.shape == v.shape,
           "q, k [N, H, d_k]; v, o [N, H, d_v]")
     N, H, d_k = q.shape
@@ -363,9 +387,10 @@ def gdn_decode_packed_into(q, k, v, g, beta, ps: PackedState, o, stream=None) ->
     _need(ps.shape == (N, H, d_k, d_v) and ps.codes.dtype == torch.uint8 and
           tuple(ps.scales.shape) == _scales_shape(N, H, d_k, d_v, ps.qdq),
           "packed state does not match the call")
-    s = lib.gdn_decode_packed(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(ps.codes),
-                              _ptr(ps.scales), N, H, d_k, d_v, GDN_DTYPE[q.dtype], GDN_GATE[gk],
-                              GDN_QDQ[ps.qdq], _ptr(o), _stream(stream))
+    with torch.cuda.device(dev):
+        s = lib.gdn_decode_packed(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(ps.codes),
+                                  _ptr(ps.scales), N, H, d_k, d_v, GDN_DTYPE[q.dtype], GDN_GATE[gk],
+                                  GDN_QDQ[ps.qdq], _ptr(o), _stream(stream, dev))
     if s != 0:
         raise GdnError(s, "gdn_decode_packed")
 

@@ -15,6 +15,7 @@
 #include "gdn_decode.cuh"
 #include "gdn_prefill_simt.cuh"
 #include "gdn_prefill_pair.cuh"
+#include "gdn_prefill_wy.cuh"
 #include "gdn_prefill_tc.cuh"
 #include <stdlib.h>
 
@@ -37,6 +38,19 @@ gdn_status err_word(unsigned **out) {
   }
   *out = g_err_ptr[dev];
   return GDN_OK;
+}
+
+// Limit of the tensor-core kernels' bounded waits: 2 s, or the value of
+// GDN_WAIT_LIMIT_NS (nanoseconds, read at every launch; 0 gives up at the
+// first wait that is not already complete).  A shorter limit exists to
+// exercise the kernels' timeout path: the kernel records GDN_ERR_TIMEOUT
+// in the error word and exits cleanly.
+uint64_t wait_limit_ns() {
+  const char *e = getenv("GDN_WAIT_LIMIT_NS");
+  if (!e || !*e) return 2000000000ull;
+  char *end = nullptr;
+  const unsigned long long v = strtoull(e, &end, 10);
+  return (end && *end == 0) ? (uint64_t)v : 2000000000ull;
 }
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -255,7 +269,8 @@ gdn_status launch_tc_one(const CUtensorMap &mq, const CUtensorMap &mk, const CUt
                            (int)gdn::tc::kSmemBytes) != cudaSuccess)
     return GDN_ERR_CUDA;
   kern<<<blocks, gdn::tc::kThreads, gdn::tc::kSmemBytes, st>>>(mq, mk, mv, mo, g, beta, state_in,
-                                                               cu, T, H, scale, o, state_out, err);
+                                                               cu, T, H, scale, o, state_out, err,
+                                                               wait_limit_ns());
   return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
@@ -273,7 +288,22 @@ gdn_status launch_pair_one(const CUtensorMap &mq, const CUtensorMap &mk, const C
                            (int)gdn::pair::kSmemBytes) != cudaSuccess)
     return GDN_ERR_CUDA;
   kern<<<2 * units, gdn::pair::kThreads, gdn::pair::kSmemBytes, st>>>(
-      mq, mk, mv, mo, g, beta, state_in, cu, T, H, scale, o, state_out, err);
+      mq, mk, mv, mo, g, beta, state_in, cu, T, H, scale, o, state_out, err, wait_limit_ns());
+  return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+// The WY-form pair (FP8 tiles): the producer CTA also forms W and hands it
+// over; the chain CTA keeps the state transposed in TMEM.
+gdn_status launch_wy_one(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv_sw,
+                         const float *g, const float *beta, const float *state_in,
+                         const int32_t *cu, int T, int H, float scale, __nv_bfloat16 *o,
+                         float *state_out, unsigned *err, unsigned units, cudaStream_t st) {
+  auto kern = gdn::wy::prefill_wy_kernel;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)gdn::wy::kSmemBytes) != cudaSuccess)
+    return GDN_ERR_CUDA;
+  kern<<<2 * units, gdn::wy::kThreads, gdn::wy::kSmemBytes, st>>>(
+      mq, mk, mv_sw, g, beta, state_in, cu, T, H, scale, o, state_out, err, wait_limit_ns());
   return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
@@ -317,6 +347,15 @@ bool use_pair(long long units) {
   return units <= slots;
 }
 
+// Among the pair kernels, FP8-tile codecs take the WY-form pair when
+// GDN_PREFILL_WY=1 in the environment (read at every call); otherwise the
+// delta-form pair.
+bool use_wy(int kind) {
+  if (kind != gdn::kQdqFp8Tile) return false;
+  const char *e = getenv("GDN_PREFILL_WY");
+  return e && e[0] == '1' && e[1] == 0;
+}
+
 // bf16 GDN at d_k = d_v = 128 runs on the tensor cores; fp32 inputs (whose
 // 1e-5 tolerance the fp16 operand splits cannot promise), per-key (KDA)
 // gates and d = 64 run on the CUDA-core kernel.
@@ -345,6 +384,12 @@ gdn_status launch_prefill_tc(const void *q, const void *k, const void *v, const 
   if ((s = make_token_map(&mo, o, H, rows, true)) != GDN_OK) return s;
   if (use_pair(blocks)) {
     if (blocks > 0x3fffffffLL) return GDN_ERR_UNSUPPORTED;
+    if (use_wy(kind)) {
+      CUtensorMap mvs;  // V tiles 128B-swizzled: the A operand of U^T = V^T (T diag(beta))^T
+      if ((s = make_token_map(&mvs, v, H, rows, true)) != GDN_OK) return s;
+      return launch_wy_one(mq, mk, mvs, g, beta, state_in, cu, T, H, scale, oo, state_out, err,
+                           nb, st);
+    }
 #define GDN_TP(QK, GR) \
   launch_pair_one<QK, GR>(mq, mk, mv, mo, g, beta, state_in, cu, T, H, scale, oo, state_out, err, nb, st)
     if (kind == gdn::kQdqNone) return GDN_TP(gdn::kQdqNone, 32);
@@ -663,14 +708,19 @@ gdn_status gdn_prefill_backward_static(const void *q, const void *k, const void 
                               dv, dg, dbeta, dstate_in, cuda_stream);
 }
 
-int gdn_prefill_schedule(int n_seq, int H, int d_k, int d_v, gdn_dtype dt, gdn_gate_kind gk) {
+int gdn_prefill_schedule(int n_seq, int H, int d_k, int d_v, gdn_dtype dt, gdn_gate_kind gk,
+                         gdn_qdq_mode qdq) {
   if (n_seq < 0 || H <= 0) return -1;
   if ((d_k != 64 && d_k != 128) || (d_v != 64 && d_v != 128)) return -1;
   if (dt != GDN_DTYPE_BF16 && dt != GDN_DTYPE_F32) return -1;
   if (gk != GDN_GATE_SCALAR && gk != GDN_GATE_PER_KEY) return -1;
+  int kind = 0, group = 32;
+  if ((unsigned)qdq > (unsigned)GDN_QDQ_INT8_GROUP64 || !qdq_params(qdq, d_v, &kind, &group))
+    return -1;
   if (!tc_path(dt, gk, d_k, d_v)) return GDN_PREFILL_CUDA_CORES;
   const long long units = (long long)n_seq * H;
-  return use_pair(units) ? GDN_PREFILL_TC_CTA_PAIR : GDN_PREFILL_TC_ONE_CTA;
+  if (!use_pair(units)) return GDN_PREFILL_TC_ONE_CTA;
+  return use_wy(kind) ? GDN_PREFILL_TC_WY_PAIR : GDN_PREFILL_TC_CTA_PAIR;
 }
 
 gdn_status gdn_last_error(void *cuda_stream) {

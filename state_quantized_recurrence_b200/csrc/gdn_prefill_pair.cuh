@@ -109,20 +109,22 @@ struct SmallC {
   int qk_pend[2], v_pend;
   int rx_pend;  // 1 + parity of an armed transfer not yet waited for
   uint32_t tmem;
-  uint64_t bar_qk[2], bar_v, bar_m2, bar_m3, bar_m4, rx_full;
+  uint64_t wait_ns;  // limit of the bounded waits (the drains keep kWaitNs)
+  uint64_t bar_qk[2], bar_v, bar_m2, bar_m3, bar_m4, rx_full, bar_drain[2];
 };
 struct SmallP {
   Gates gt;
   int abort;
   int qk_pend[2];
   uint32_t tmem;
-  uint64_t bar_qk[2], bar_m1, rx_free;
+  uint64_t wait_ns;
+  uint64_t bar_qk[2], bar_m1, rx_free, bar_drain[2];
 };
 static_assert(sizeof(SmallC) <= kSmallBytes && sizeof(SmallP) <= kSmallBytes, "small blocks");
 
 template <class S>
 __device__ __forceinline__ bool wait_local(uint64_t *bar, uint32_t parity, S *sm, unsigned *err) {
-  if (!sm100::mbar_wait(bar, parity, kWaitNs)) {
+  if (!sm100::mbar_wait(bar, parity, sm->wait_ns)) {
     sm->abort = 1;
     atomicOr(err, kErrTimeout);
     return false;
@@ -131,7 +133,7 @@ __device__ __forceinline__ bool wait_local(uint64_t *bar, uint32_t parity, S *sm
 }
 template <class S>
 __device__ __forceinline__ bool wait_cluster(uint64_t *bar, uint32_t parity, S *sm, unsigned *err) {
-  if (!sm100::mbar_wait_cluster(bar, parity, kWaitNs)) {
+  if (!sm100::mbar_wait_cluster(bar, parity, sm->wait_ns)) {
     sm->abort = 1;
     atomicOr(err, kErrTimeout);
     return false;
@@ -147,7 +149,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     const float *__restrict__ beta, const float *__restrict__ state_in,
                     const int *__restrict__ cu_seqlens, int T, int H, float scale,
                     __nv_bfloat16 *__restrict__ o, float *__restrict__ state_out,
-                    unsigned *__restrict__ err) {
+                    unsigned *__restrict__ err, uint64_t wait_ns) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = sm100::smem_u32(smem_raw);
   const uint32_t base = (raw_addr + 1023u) & ~1023u;
@@ -213,8 +215,11 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       sm100::mbar_init(&smc->bar_m3, 1);
       sm100::mbar_init(&smc->bar_m4, 1);
       sm100::mbar_init(&smc->rx_full, 1);
+      sm100::mbar_init(&smc->bar_drain[0], 1);
+      sm100::mbar_init(&smc->bar_drain[1], 1);
       sm100::fence_mbar_init();
       smc->abort = 0;
+      smc->wait_ns = wait_ns;
       smc->exact = 0;
       smc->qk_pend[0] = smc->qk_pend[1] = smc->v_pend = 0;
       // chunk 0's transfer (issued only after the cluster barrier below)
@@ -232,8 +237,11 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       sm100::mbar_init(&smp->bar_qk[1], 1);
       sm100::mbar_init(&smp->bar_m1, 1);
       sm100::mbar_init(&smp->rx_free, 1);
+      sm100::mbar_init(&smp->bar_drain[0], 1);
+      sm100::mbar_init(&smp->bar_drain[1], 1);
       sm100::fence_mbar_init();
       smp->abort = 0;
+      smp->wait_ns = wait_ns;
       smp->qk_pend[0] = smp->qk_pend[1] = 0;
     }
     if (warp == 0) {
@@ -294,7 +302,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       sm100::tc_fence_after();
       if (ok) issue_mma1(0);
     }
-    for (int j = 0; j < n_chunks && !sm->abort; ++j) {
+    for (int j = 0; j < n_chunks; ++j) {  // left only at the checks after barriers
       const int n = chunk_len(j);
       const int b = j & 1;
       const uint32_t stg = base + P_STG + (uint32_t)b * kRxBytes;
@@ -616,7 +624,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     long long tb_prev = 0;
     int n_prev = 0;
     float hs_prev = 1.0f;
-    for (int it = 0; it < n_chunks && !sm->abort; ++it) {
+    for (int it = 0; it < n_chunks; ++it) {  // left only at the checks after barriers
       const long long c0 = (long long)it * kC;
       const int n = chunk_len(it);
       const long long tb = t0 + c0;
@@ -886,8 +894,14 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     }
   }
 
-  // ---- teardown: neither CTA leaves while the peer may still copy into or
+  // ---- teardown: an aborted CTA lets the MMAs of its issuing warps (0 and
+  //      4) finish; neither CTA leaves while the peer may still copy into or
   //      arrive on its shared memory ----
+  {
+    const int ab = rank == 0 ? smc->abort : smp->abort;
+    uint64_t *bd = rank == 0 ? smc->bar_drain : smp->bar_drain;
+    if (ab && (warp == 0 || warp == 4)) drain_mmas(&bd[warp >> 2]);
+  }
   sm100::tc_fence_before();
   __syncthreads();
   sm100::cluster_sync();

@@ -99,7 +99,8 @@ struct Small {
   int abort;
   int qk_pend[2], v_pend;  // 1 + parity of an issued, unconsumed TMA phase
   uint32_t tmem;
-  uint64_t bar_qk[2], bar_v, bar_m1, bar_m2, bar_m3, bar_m4;
+  uint64_t wait_ns;  // limit of the bounded waits (the drains keep kWaitNs)
+  uint64_t bar_qk[2], bar_v, bar_m1, bar_m2, bar_m3, bar_m4, bar_drain[2];
 };
 static_assert(sizeof(Small) <= 4096, "small-state block overflows its slot");
 static_assert(sizeof(Gates) % 16 == 0 && OFF_SMALL % 16 == 0, "gate arrays must stay 16-byte aligned");
@@ -108,7 +109,7 @@ static_assert(OFF_P % 16 == 0 && OFF_T % 16 == 0 && (LDT * 4) % 16 == 0, "float4
 // Bounded wait by every calling thread; a timeout marks the CTA aborted.
 __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, Small *sm,
                                               unsigned *err) {
-  if (!sm100::mbar_wait(bar, parity, kWaitNs)) {
+  if (!sm100::mbar_wait(bar, parity, sm->wait_ns)) {
     sm->abort = 1;
     atomicOr(err, kErrTimeout);
     return false;
@@ -124,7 +125,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                   const float *__restrict__ beta, const float *__restrict__ state_in,
                   const int *__restrict__ cu_seqlens, int T, int H, float scale,
                   __nv_bfloat16 *__restrict__ o, float *__restrict__ state_out,
-                  unsigned *__restrict__ err) {
+                  unsigned *__restrict__ err, uint64_t wait_ns) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = sm100::smem_u32(smem_raw);
   const uint32_t base = (raw_addr + 1023u) & ~1023u;
@@ -176,8 +177,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     sm100::mbar_init(&sm->bar_m2, 1);
     sm100::mbar_init(&sm->bar_m3, 1);
     sm100::mbar_init(&sm->bar_m4, 1);
+    sm100::mbar_init(&sm->bar_drain[0], 1);
+    sm100::mbar_init(&sm->bar_drain[1], 1);
     sm100::fence_mbar_init();
     sm->abort = 0;
+    sm->wait_ns = wait_ns;
     sm->exact = 0;
     sm->qk_pend[0] = sm->qk_pend[1] = sm->v_pend = 0;
   }
@@ -298,7 +302,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   };
 
   int it = 0;
-  for (long long c0 = 0; c0 < L && !sm->abort; c0 += kC, ++it) {
+  for (long long c0 = 0; c0 < L; c0 += kC, ++it) {  // left only at the checks after barriers
     const int n = (int)min((long long)kC, L - c0);
     const long long tb = t0 + c0;
     const bool last = it == n_chunks - 1;
@@ -793,14 +797,16 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   flush_outputs();  // a partial last chunk's outputs
   if (tid == kStoreTid) sm100::bulk_wait_all();
 
-  // An aborted CTA lets its outstanding TMA loads land (again bounded)
-  // before its shared memory is released.
+  // An aborted CTA lets its outstanding TMA loads land and its MMAs (issued
+  // by warps 0 and 4) finish, again bounded, before its shared memory and
+  // TMEM are released.
   if (tid == 0 && sm->abort) {
     for (int b = 0; b < 2; ++b)
       if (sm->qk_pend[b])
         (void)sm100::mbar_wait(&sm->bar_qk[b], (uint32_t)(sm->qk_pend[b] - 1), kWaitNs);
     if (sm->v_pend) (void)sm100::mbar_wait(&sm->bar_v, (uint32_t)(sm->v_pend - 1), kWaitNs);
   }
+  if (sm->abort && (warp == 0 || warp == 4)) drain_mmas(&sm->bar_drain[warp >> 2]);
   __syncthreads();
   if (warp == 0) {
     sm100::tc_fence_after();

@@ -65,9 +65,11 @@ __device__ __forceinline__ uint64_t global_ns() {
 }
 
 // Bounded wait: true once the phase with `parity` completed, false when
-// `limit_ns` nanoseconds passed first.
+// `limit_ns` nanoseconds passed first (a limit of 0 gives up as soon as one
+// test finds the phase incomplete).
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
+  if (limit_ns == 0) return false;
   const uint64_t start = global_ns();
   for (;;) {
 #pragma unroll 1
@@ -111,6 +113,7 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t pa
 }
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
   if (mbar_try_wait_cluster(bar, parity)) return true;
+  if (limit_ns == 0) return false;
   const uint64_t start = global_ns();
   for (;;) {
 #pragma unroll 1

@@ -120,6 +120,18 @@ __device__ __forceinline__ void convert_kq_half(uint8_t *buf, int n, int t, int 
   }
 }
 
+// After an abort: the lane of this (converged) warp that issued its MMAs
+// makes `bar` (count 1, unused so far) track all of them and waits for them
+// (bounded, 2 s), so that no MMA still reads shared memory or writes TMEM
+// when the CTA releases both.
+__device__ __forceinline__ void drain_mmas(uint64_t *bar) {
+  if (sm100::elect_one()) {
+    sm100::mma_commit(bar);
+    (void)sm100::mbar_wait(bar, 0, 2000000000ull);
+  }
+  __syncwarp();
+}
+
 __device__ __forceinline__ uint64_t kdesc(uint32_t addr) {
   return sm100::smem_desc_sw128(addr, 16, 1024);
 }

@@ -257,11 +257,12 @@ def test_prefill_schedule_host_cases(lib):
     """Shapes off the tensor-core path choose the CUDA-core kernel without
     touching a device; shapes gdn_prefill rejects give -1."""
     I = ctypes.c_int
-    lib.gdn_prefill_schedule.argtypes = [I] * 6
+    lib.gdn_prefill_schedule.argtypes = [I] * 7
     lib.gdn_prefill_schedule.restype = I
-    assert lib.gdn_prefill_schedule(2, 4, 128, 128, 1, 0) == 0   # fp32
-    assert lib.gdn_prefill_schedule(2, 4, 128, 128, 0, 1) == 0   # KDA gates
-    assert lib.gdn_prefill_schedule(2, 4, 64, 64, 0, 0) == 0     # d = 64
-    assert lib.gdn_prefill_schedule(2, 4, 96, 128, 0, 0) == -1
-    assert lib.gdn_prefill_schedule(2, 0, 128, 128, 0, 0) == -1
-    assert lib.gdn_prefill_schedule(2, 4, 128, 128, 7, 0) == -1
+    assert lib.gdn_prefill_schedule(2, 4, 128, 128, 1, 0, 1) == 0   # fp32
+    assert lib.gdn_prefill_schedule(2, 4, 128, 128, 0, 1, 2) == 0   # KDA gates
+    assert lib.gdn_prefill_schedule(2, 4, 64, 64, 0, 0, 1) == 0     # d = 64
+    assert lib.gdn_prefill_schedule(2, 4, 96, 128, 0, 0, 1) == -1
+    assert lib.gdn_prefill_schedule(2, 0, 128, 128, 0, 0, 1) == -1
+    assert lib.gdn_prefill_schedule(2, 4, 128, 128, 7, 0, 1) == -1
+    assert lib.gdn_prefill_schedule(2, 4, 128, 128, 1, 0, 9) == -1   # no such codec

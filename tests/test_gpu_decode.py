@@ -8,8 +8,11 @@
   one-step / 1e-4 budget (tiny fp32 config, serving-decode shapes, KDA);
 * free-running without QDQ: 24 steps within the float tolerance;
 * the full serving-decode shapes (256 sequences x 32 heads, d = 128, INT8
-  g32): two teacher-forced steps, compared on a quarter of the sequences
-  (the benchmark's full 512-token run is checked by its own sampled check).
+  g32): two teacher-forced steps, compared on a quarter of the sequences;
+  and the benchmark's whole run, 512 tokens of all 256 sequences, on 8
+  sampled sequences (every head): teacher-forced at every one of the 512
+  steps, and free-running against the oracle's own chain (a looser bound:
+  see FREE_RUNNING_DECODE_CHAIN_TOL).
 """
 
 import numpy as np
@@ -18,7 +21,7 @@ import torch
 
 import gdn_synth as gs
 import oracle
-from parity import TOL, assert_flip_budget, check_codes, rel_err
+from parity import TOL, assert_flip_budget, assert_rows_close, check_codes, rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -68,6 +71,7 @@ def _teacher_forced(cuda_lib, case, S0: torch.Tensor, steps: int, label: str):
             inp["dec_q"][sl], inp["dec_k"][sl], inp["dec_v"][sl], inp["dec_g"][sl],
             inp["dec_beta"][sl], prev, per_key_gate=per_key, qdq=case.qdq, want_codes=True)
         worst_o = max(worst_o, rel_err(o.float().cpu().numpy(), o_ref[0]))
+        assert_rows_close(o.float().cpu().numpy(), o_ref[0], case.dtype, f"{label} step {t}")
         stats.append(check_codes(S.cpu().numpy(), s_ref, codes, scales, case.qdq,
                                  label=f"{label} step {t}"))
     assert worst_o <= TOL[case.dtype], (label, worst_o)
@@ -135,9 +139,69 @@ def test_decode_full_serving_shape(cuda_lib):
             inp["dec_q"][sl], inp["dec_k"][sl], inp["dec_v"][sl], inp["dec_g"][sl],
             inp["dec_beta"][sl], prev, per_key_gate=False, qdq=case.qdq, want_codes=True)
         assert rel_err(o[:64].float().cpu().numpy(), o_ref[0]) <= TOL["bf16"]
+        assert_rows_close(o[:64].float().cpu().numpy(), o_ref[0], "bf16", f"full decode {t}")
         stats.append(check_codes(S[:64].cpu().numpy(), s_ref, codes, scales, case.qdq,
                                  label=f"full decode step {t}"))
     assert_flip_budget(stats, "full serving decode")
+
+
+# Free-running over the 512-token chain, the QDQ after every token turns
+# last-bit differences into one-step code flips that persist: an fp32
+# evaluation of the same recurrence with the oracle's own codec departs
+# from the fp64 oracle by up to 1.2e-2 per token step (measured on two of
+# these sequences), so no fp32 implementation meets 2e-3 there.  The run
+# is therefore held to the teacher-forced bar at every step, and its
+# free-running distance only to 3e-2, which catches a wrong recurrence.
+FREE_RUNNING_DECODE_CHAIN_TOL = 3e-2
+
+
+def test_decode_full_serving_run(cuda_lib):
+    """The serving-decode workload as the benchmark runs it: 512 consecutive
+    single-token calls over all 256 sequences x 32 heads (INT8 g32 after
+    every token).  On 8 sequences spread over the batch: every one of the
+    512 steps teacher-forced (the oracle advances the GPU's own previous
+    state; every head's outputs, and the codes of a rotating window of 8
+    heads, within the bar), and the whole free-running chain against the
+    oracle's own 512-token chain."""
+    case = gs.CONFIGS["serving_decode"]
+    assert case.decode_steps == 512
+    inp = gs.generate(case)
+    S = inp["state_in"].clone().cuda()
+    dq, dk, dv = (inp[x].cuda() for x in ("dec_q", "dec_k", "dec_v"))
+    dg, db = inp["dec_g"].cuda(), inp["dec_beta"].cuda()
+    o = torch.empty(dv.shape, dtype=dq.dtype, device="cuda")
+    seqs = [0, 37, 73, 110, 146, 183, 219, 255]
+    stats, worst_tf = [], 0.0
+    for t in range(case.decode_steps):
+        prev = S[seqs].cpu().numpy()
+        cuda_lib.gdn_decode_into(dq[t], dk[t], dv[t], dg[t], db[t], S, o[t], qdq=case.qdq)
+        sl = (slice(t, t + 1), seqs)
+        o_ref, s_ref, codes, scales = oracle.decode(
+            inp["dec_q"][sl], inp["dec_k"][sl], inp["dec_v"][sl], inp["dec_g"][sl],
+            inp["dec_beta"][sl], prev, per_key_gate=False, qdq=case.qdq, want_codes=True)
+        o_g = o[t, seqs].float().cpu().numpy()
+        worst_tf = max(worst_tf, rel_err(o_g, o_ref[0]))
+        assert_rows_close(o_g, o_ref[0], "bf16", f"serving run step {t}")
+        # codes of 8 of the 32 heads per step, a window that rotates over
+        # the heads (all heads every 4 steps), to keep the check fast
+        hs = [(8 * t + i) % case.H for i in range(8)]
+        stats.append(check_codes(S[seqs][:, hs].cpu().numpy(), s_ref[:, hs], codes[:, hs],
+                                 scales[:, hs], case.qdq, label=f"serving run step {t}"))
+    cuda_lib.check_last_error(where="serving decode run")
+    assert worst_tf <= TOL["bf16"], worst_tf
+    assert_flip_budget(stats, "serving decode, 512 steps")
+
+    sl = (slice(None), seqs)
+    o_ref, s_ref = oracle.decode(inp["dec_q"][sl], inp["dec_k"][sl], inp["dec_v"][sl],
+                                 inp["dec_g"][sl], inp["dec_beta"][sl], inp["state_in"][seqs],
+                                 per_key_gate=False, qdq=case.qdq)
+    o_g = o[:, seqs].float().cpu().numpy()
+    worst_step = max(rel_err(o_g[t], o_ref[t]) for t in range(case.decode_steps))
+    assert worst_step <= FREE_RUNNING_DECODE_CHAIN_TOL, worst_step
+    s_g = S[seqs].cpu().numpy()
+    worst_unit = max(rel_err(s_g[i, h], s_ref[i, h]) for i in range(len(seqs))
+                     for h in range(case.H))
+    assert worst_unit <= FREE_RUNNING_DECODE_CHAIN_TOL, worst_unit
 
 
 def test_decode_single_head_edge(cuda_lib):

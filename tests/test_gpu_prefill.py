@@ -10,7 +10,11 @@
   every chunk boundary matches outputs and codes;
 * the five workloads: the tiny one in full, reduced copies of the others,
   and the full-size prefill workloads in the benchmark's launch
-  configuration compared on sampled (sequence, head) units;
+  configuration: 16 sampled (sequence, head) units each, free-running over
+  their whole sequences and teacher-forced on 8 or more chunks per unit;
+  the packed workload's 32-token decode tail for every (sequence, head);
+* INT8 groups of 16, 32 and 64 on the tensor-core kernels over several
+  chunks from random states;
 * edge cases: empty sequences, an all-empty packed batch, a malformed
   cu_seqlens reported through gdn_last_error, state_out aliasing state_in.
 
@@ -18,27 +22,37 @@ Every test runs three times: under the automatic schedule choice and with
 the single-CTA and the CTA-pair tensor-core kernels forced.
 """
 
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
 
 import gdn_synth as gs
 import oracle
-from parity import TOL, assert_flip_budget, check_codes, per_unit_rel_err, rel_err
+from parity import (TOL, assert_flip_budget, assert_rows_close, check_codes,
+                    per_unit_rel_err, rel_err)
 
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(autouse=True, params=["auto", "single", "pair"])
+@pytest.fixture(autouse=True, params=["auto", "single", "pair", "wy"])
 def schedule(request, monkeypatch):
     """Every case under the library's own choice of tensor-core schedule and
-    under each schedule forced (GDN_PREFILL_CTA_PAIR): one CTA per
-    (sequence, head), or a CTA pair.  Cases off the tensor-core path (fp32,
-    KDA gates, d = 64) run the same kernel in all three."""
+    under each schedule forced: one CTA per (sequence, head)
+    (GDN_PREFILL_CTA_PAIR=0), the delta-form CTA pair (GDN_PREFILL_CTA_PAIR=1),
+    or the WY-form pair (GDN_PREFILL_CTA_PAIR=1, GDN_PREFILL_WY=1: FP8 tiles;
+    other codecs keep the delta-form pair).  Cases off the tensor-core path
+    (fp32, KDA gates, d = 64) run the same kernel in all four."""
+    monkeypatch.delenv("GDN_PREFILL_WY", raising=False)
     if request.param == "auto":
         monkeypatch.delenv("GDN_PREFILL_CTA_PAIR", raising=False)
+    elif request.param == "single":
+        monkeypatch.setenv("GDN_PREFILL_CTA_PAIR", "0")
     else:
-        monkeypatch.setenv("GDN_PREFILL_CTA_PAIR", "1" if request.param == "pair" else "0")
+        monkeypatch.setenv("GDN_PREFILL_CTA_PAIR", "1")
+        if request.param == "wy":
+            monkeypatch.setenv("GDN_PREFILL_WY", "1")
     return request.param
 
 
@@ -82,6 +96,7 @@ def test_prefill_free_running_no_qdq_packed(cuda_lib, gate, dtype, dk, dv):
     o, s = run_gpu(cuda_lib, inp, case)
     o_ref, s_ref = oracle.prefill(inp, case)
     assert rel_err(o, o_ref.reshape(o.shape)) <= TOL[dtype]
+    assert_rows_close(o, o_ref, dtype, "free-running packed o")
     assert per_unit_rel_err(s, s_ref, axes=(-2, -1)) <= TOL[dtype]
 
 
@@ -93,6 +108,7 @@ def test_prefill_free_running_no_qdq_dense(cuda_lib, gate):
     o, s = run_gpu(cuda_lib, inp, case)
     o_ref, s_ref = oracle.prefill(inp, case)
     assert rel_err(o, o_ref.reshape(o.shape)) <= TOL["bf16"]
+    assert_rows_close(o, o_ref, "bf16", "free-running dense o")
     assert per_unit_rel_err(s, s_ref, axes=(-2, -1)) <= TOL["bf16"]
 
 
@@ -124,6 +140,7 @@ def teacher_forced_chunks(cuda_lib, case, label):
                 sub["q"], sub["k"], sub["v"], sub["g"], sub["beta"], st, cu,
                 per_key_gate=per_key, qdq=case.qdq, want_codes=True)
             worst_o = max(worst_o, rel_err(o_c[0], o_r))
+            assert_rows_close(o_c[0], o_r, case.dtype, f"{label} seq {si} chunk {c0 // 64}")
             if case.qdq != "none":
                 stats.append(check_codes(s_c, s_r, codes, scales, case.qdq,
                                          label=f"{label} seq {si} chunk {c0 // 64}"))
@@ -166,73 +183,218 @@ def test_prefill_teacher_forced(cuda_lib, base, over):
     teacher_forced_chunks(cuda_lib, case, f"{base} {over}")
 
 
-def _sampled_units(cuda_lib, case, units, tf_units):
-    """Full workload on the GPU; free-running comparison on `units`
-    (seq, head) pairs and a teacher-forced last chunk on `tf_units`."""
+_TENSORS = ("q", "k", "v", "g", "beta")
+
+
+def _flat(inp):
+    return {x: inp[x].reshape((-1,) + inp[x].shape[2:]) for x in _TENSORS}
+
+
+def _unit_batch(inp, units, ranges):
+    """Oracle inputs for (sequence, head) units over token ranges [a, b) of
+    their sequences: every unit becomes one packed sequence of one head."""
+    starts = np.concatenate([[0], np.cumsum(inp["lengths"])])
+    flat = _flat(inp)
+    parts = {x: [] for x in _TENSORS}
+    cu = [0]
+    for (si, h), (a, b) in zip(units, ranges):
+        sl = slice(int(starts[si] + a), int(starts[si] + b))
+        for x in _TENSORS:
+            parts[x].append(flat[x][sl][:, h:h + 1])
+        cu.append(cu[-1] + (b - a))
+    return {x: torch.cat(parts[x]) for x in _TENSORS}, np.array(cu, dtype=np.int32)
+
+
+def _unit_states(S, units, dk, dv):
+    """[n_units, 1, d_k, d_v] states of the units from [n_seq, H, ...] (None: zero)."""
+    if S is None:
+        return torch.zeros((len(units), 1, dk, dv))
+    S = torch.as_tensor(S)
+    return torch.stack([S[si, h:h + 1] for (si, h) in units])
+
+
+def _truncated(inp, case, lens):
+    """The workload cut to the first lens[s] tokens of every sequence: a
+    dense batch when the case is dense and the cut uniform (the layout the
+    benchmark runs), otherwise a packed batch of the same sequences."""
+    if inp["cu_seqlens"] is None and len(set(lens)) == 1:
+        sub = {x: inp[x][:, :lens[0]].contiguous() for x in _TENSORS}
+        sub.update(state_in=inp["state_in"], cu_seqlens=None, lengths=list(lens))
+        return sub, dataclasses.replace(case, T=int(lens[0]))
+    starts = np.concatenate([[0], np.cumsum(inp["lengths"])])
+    flat = _flat(inp)
+    sub = {x: torch.cat([flat[x][int(starts[si]):int(starts[si] + n)]
+                         for si, n in enumerate(lens)])[None] for x in _TENSORS}
+    cu = torch.zeros(len(lens) + 1, dtype=torch.int32)
+    cu[1:] = torch.cumsum(torch.tensor(lens, dtype=torch.int64), 0).to(torch.int32)
+    sub.update(state_in=inp["state_in"], cu_seqlens=cu, lengths=list(lens))
+    return sub, dataclasses.replace(case, lengths=tuple(int(n) for n in lens), varlen_max=0, T=0)
+
+
+def _check_full_workload(cuda_lib, case, units, n_tf_chunks=8):
+    """The whole workload in one call, as the benchmark launches it, then:
+
+    * free-running: the oracle over every sampled (sequence, head) unit's
+      whole sequence, from the same initial state; o and the final state
+      norm-wise per unit;
+    * teacher-forced: for each sampled unit, ``n_tf_chunks`` chunks spread
+      over its sequence (first, second and last included).  The GPU's state
+      at the start of chunk c is the final state of the same workload cut
+      to its first 64 c tokens per sequence (the same kernel computes the
+      same chunks bit for bit), and the state after it that of the cut at
+      64 (c + 1); the oracle restarted from the former over chunk c must
+      give the latter's codes (one-step flips within the budget) and the
+      single call's outputs of that chunk (norm-wise and per element)."""
     inp = gs.generate(case)
     o, s = run_gpu(cuda_lib, inp, case)
-    lengths = inp["lengths"]
+    lengths = [int(x) for x in inp["lengths"]]
     starts = np.concatenate([[0], np.cumsum(lengths)])
-    H, dv = case.H, case.d_v
+    H, dk, dv = case.H, case.d_k, case.d_v
     per_key = case.gate == "per_key"
-    flat = {x: inp[x].reshape((-1,) + inp[x].shape[2:]) for x in ("q", "k", "v", "g", "beta")}
     o_flat = o.reshape((-1, H, dv))
-    stats = []
-    for (si, h) in units:
-        sl = slice(int(starts[si]), int(starts[si + 1]))
-        st = None if inp["state_in"] is None else inp["state_in"][si:si + 1, h:h + 1]
-        cu = np.array([0, lengths[si]], dtype=np.int32)
-        args = [flat[x][sl][:, h:h + 1] for x in ("q", "k", "v", "g", "beta")]
-        o_r, s_r = oracle.recurrence(*args, st, cu, per_key_gate=per_key, qdq=case.qdq)
-        assert rel_err(o_flat[sl, h], o_r[:, 0]) <= TOL[case.dtype], (si, h)
-        assert rel_err(s[si, h], s_r[0, 0]) <= TOL[case.dtype], (si, h)
-    for si in tf_units:
-        L = lengths[si]
-        if L <= 64:
-            continue
-        cut = ((L - 1) // 64) * 64
-        sl = slice(int(starts[si]), int(starts[si] + cut))
-        sub = {x: flat[x][sl][None] for x in ("q", "k", "v", "g", "beta")}
-        sub["state_in"] = None if inp["state_in"] is None else inp["state_in"][si:si + 1]
-        sub["cu_seqlens"] = None
-        _, s_mid = run_gpu(cuda_lib, sub, gs.Case("p", n_seq=1, H=H, d_k=case.d_k, d_v=dv, T=cut,
-                                                  dtype=case.dtype, gate=case.gate, qdq=case.qdq))
-        sl2 = slice(int(starts[si] + cut), int(starts[si + 1]))
-        args = [flat[x][sl2] for x in ("q", "k", "v", "g", "beta")]
-        cu = np.array([0, L - cut], dtype=np.int32)
-        o_r, s_r, codes, scales = oracle.recurrence(*args, s_mid, cu, per_key_gate=per_key,
-                                                    qdq=case.qdq, want_codes=True)
-        assert rel_err(o_flat[sl2], o_r) <= TOL[case.dtype]
-        stats.append(check_codes(s[si:si + 1], s_r, codes, scales, case.qdq,
-                                 label=f"{case.name} seq {si} last chunk"))
-    return assert_flip_budget(stats, case.name)
+    tol = TOL[case.dtype]
+
+    # free-running, all sampled units in one oracle call
+    batch, cu = _unit_batch(inp, units, [(0, lengths[si]) for si, _ in units])
+    o_r, s_r = oracle.recurrence(*(batch[x] for x in _TENSORS),
+                                 _unit_states(inp["state_in"], units, dk, dv), cu,
+                                 per_key_gate=per_key, qdq=case.qdq)
+    for i, (si, h) in enumerate(units):
+        o_u = o_flat[int(starts[si]):int(starts[si + 1]), h]
+        assert rel_err(o_u, o_r[cu[i]:cu[i + 1], 0]) <= tol, ("o", si, h)
+        assert rel_err(s[si, h], s_r[i, 0]) <= tol, ("state", si, h)
+
+    # teacher-forced, n_tf_chunks chunk positions per sequence
+    n_ch = [(L + 63) // 64 for L in lengths]
+    pos = [sorted({0, min(1, n - 1)} | {round(j * (n - 1) / (n_tf_chunks - 1))
+                                        for j in range(n_tf_chunks)}) if n else []
+           for n in n_ch]
+    n_pos = max(len(p) for p in pos)
+    stats, checked = [], 0
+    for j in range(n_pos):
+        c_of = [p[j] if j < len(p) else (p[-1] if p else 0) for p in pos]
+        before = [min(64 * c, L) for c, L in zip(c_of, lengths)]
+        after = [min(64 * (c + 1), L) for c, L in zip(c_of, lengths)]
+        if max(before) == 0:
+            S0 = (inp["state_in"].numpy() if inp["state_in"] is not None
+                  else np.zeros((case.n_seq, H, dk, dv), np.float32))
+        else:
+            sub, sc = _truncated(inp, case, before)
+            _, S0 = run_gpu(cuda_lib, sub, sc)
+        sub, sc = _truncated(inp, case, after)
+        _, S1 = run_gpu(cuda_lib, sub, sc)
+        live = [(si, h) for (si, h) in units if after[si] > before[si]]
+        batch, cu = _unit_batch(inp, live, [(before[si], after[si]) for si, _ in live])
+        o_t, s_t, codes, scales = oracle.recurrence(
+            *(batch[x] for x in _TENSORS), _unit_states(S0, live, dk, dv), cu,
+            per_key_gate=per_key, qdq=case.qdq, want_codes=True)
+        for i, (si, h) in enumerate(live):
+            sl = slice(int(starts[si] + before[si]), int(starts[si] + after[si]))
+            ref = o_t[cu[i]:cu[i + 1], 0]
+            assert rel_err(o_flat[sl, h], ref) <= tol, ("tf o", si, h, c_of[si])
+            assert_rows_close(o_flat[sl, h], ref, case.dtype, f"tf o {si} {h} {c_of[si]}")
+        if case.qdq != "none":
+            got = np.stack([S1[si, h:h + 1] for (si, h) in live])
+            stats.append(check_codes(got, s_t, codes, scales, case.qdq,
+                                     label=f"{case.name} position {j}"))
+        checked += len(live)
+    assert checked >= n_tf_chunks * len(units)
+    return assert_flip_budget(stats, case.name) if stats else None
 
 
 def test_full_gdn_prefill_workload(cuda_lib):
+    """B=4, H=16, T=4096, FP8 tiles: 16 of the 64 units, 9 chunks each."""
     case = gs.CONFIGS["gdn_prefill"]
-    _sampled_units(cuda_lib, case, units=[(0, 0), (1, 7), (2, 15), (3, 3)], tf_units=[0, 3])
+    units = [(si, h) for si in range(4) for h in (0, 5, 10, 15)]
+    _check_full_workload(cuda_lib, case, units)
 
 
 def test_full_kda_prefill_workload(cuda_lib):
+    """B=2, H=32, T=8192, per-key gates, INT8 g32: 16 of the 64 units."""
     case = gs.CONFIGS["kda_prefill"]
-    _sampled_units(cuda_lib, case, units=[(0, 0), (1, 31), (0, 17)], tf_units=[1])
+    units = [(si, h) for si in range(2) for h in range(0, 32, 4)]
+    _check_full_workload(cuda_lib, case, units)
+
+
+def _varlen_units(lengths, n=16):
+    """n units of distinct sequences with at least 9 chunks, spread over
+    the length range and the heads."""
+    order = [int(i) for i in np.argsort(lengths) if lengths[i] > 8 * 64]
+    pick = [order[round(j * (len(order) - 1) / (n - 1))] for j in range(n)]
+    assert len(set(pick)) == n
+    return [(si, (3 * j) % 16) for j, si in enumerate(pick)]
 
 
 def test_full_varlen_workload(cuda_lib):
-    case = gs.CONFIGS["varlen"]
-    inp_len = gs.generate(gs.small_case("varlen", decode_steps=0))["lengths"]
-    order = np.argsort(inp_len)
-    units = [(int(order[0]), 0), (int(order[-1]), 15), (int(order[31]), 5), (int(order[-2]), 9)]
-    _sampled_units(cuda_lib, gs.small_case("varlen", decode_steps=0), units=units,
-                   tf_units=[int(order[-1]), int(order[40])])
+    """64 packed sequences of U{1..4096} tokens, H=16, random states, FP8
+    tiles (1,024 units): 16 units, 8 or more chunks each."""
+    case = gs.small_case("varlen", decode_steps=0)
     assert case.n_seq == 64
+    lengths = gs.generate(case)["lengths"]
+    _check_full_workload(cuda_lib, case, _varlen_units(lengths))
+
+
+def test_full_varlen_workload_decode_tail(cuda_lib, schedule):
+    """The packed workload end to end: the packed prefill of all 64
+    sequences, then 32 decode tokens for every sequence (FP8 tiles, the
+    prefill's codec) starting from the GPU's own prefill states; every
+    decode step of every (sequence, head) is compared with the oracle
+    restarted from the GPU's state before it (outputs of all 1,024 units;
+    codes within the one-step / 1e-4 budget for a window of 256 units that
+    rotates over all of them every 4 steps).  Run under the automatic
+    schedule and the WY-form pair (the decode kernel is the same in all)."""
+    if schedule not in ("auto", "wy"):
+        pytest.skip("the decode tail is the same kernel under every prefill schedule")
+    case = gs.CONFIGS["varlen"]
+    assert case.decode_steps == 32
+    inp = gs.generate(case)
+    _, st = run_gpu(cuda_lib, inp, case)
+    S = torch.from_numpy(st).cuda()
+    stats, worst_o = [], 0.0
+    for t in range(case.decode_steps):
+        prev = S.cpu().numpy().copy()
+        o = cuda_lib.gdn_decode(dev(inp["dec_q"][t]), dev(inp["dec_k"][t]), dev(inp["dec_v"][t]),
+                                dev(inp["dec_g"][t]), dev(inp["dec_beta"][t]), S, qdq=case.qdq)
+        torch.cuda.synchronize()
+        sl = slice(t, t + 1)
+        o_ref, s_ref, codes, scales = oracle.decode(
+            inp["dec_q"][sl], inp["dec_k"][sl], inp["dec_v"][sl], inp["dec_g"][sl],
+            inp["dec_beta"][sl], prev, per_key_gate=False, qdq=case.qdq, want_codes=True)
+        o_g = o.float().cpu().numpy()
+        worst_o = max(worst_o, rel_err(o_g, o_ref[0]))
+        assert_rows_close(o_g, o_ref[0], "bf16", f"decode tail step {t}")
+        # units (sequence, head) flattened; 256 of the 1,024 per step
+        win = (256 * t + np.arange(256)) % (case.n_seq * case.H)
+        si, hi = win // case.H, win % case.H
+        S_h = S.cpu().numpy()
+        stats.append(check_codes(S_h[si, hi][:, None], s_ref[si, hi][:, None],
+                                 codes[si, hi][:, None], scales[si, hi][:, None], case.qdq,
+                                 label=f"decode tail step {t}"))
+    assert worst_o <= TOL["bf16"], worst_o
+    assert_flip_budget(stats, "varlen decode tail")
 
 
 def test_long_single_sequence(cuda_lib):
     """One sequence of 16384 tokens (256 chunks), one head."""
     case = gs.Case("long", n_seq=1, H=1, d_k=128, d_v=128, T=16384, dtype="bf16",
                    gate="scalar", qdq="fp8_tile64", state="normal", seed=81)
-    _sampled_units(cuda_lib, case, units=[(0, 0)], tf_units=[0])
+    _check_full_workload(cuda_lib, case, units=[(0, 0)], n_tf_chunks=12)
+
+
+@pytest.mark.parametrize("mode", ["int8_g32", "int8_g16", "int8_g64"])
+def test_prefill_int8_tensor_cores_multichunk(cuda_lib, mode):
+    """bf16 GDN at d = 128 takes the tensor-core kernels for every codec: INT8
+    groups of 32, 16 and 64 over 6 chunks (a partial last one) from random
+    initial states (whose hi/lo split path an INT8 state keeps), free-running
+    against the oracle and teacher-forced chunk by chunk."""
+    case = gs.Case("int8tc", n_seq=2, H=3, d_k=128, d_v=128, T=5 * 64 + 21, dtype="bf16",
+                   gate="scalar", qdq=mode, state="normal", seed=95)
+    inp = gs.generate(case)
+    o, s = run_gpu(cuda_lib, inp, case)
+    o_ref, s_ref = oracle.prefill(inp, case)
+    assert rel_err(o, o_ref.reshape(o.shape)) <= TOL["bf16"]
+    assert per_unit_rel_err(s, s_ref, axes=(-2, -1)) <= TOL["bf16"]
+    teacher_forced_chunks(cuda_lib, case, f"int8 tensor cores {mode}")
 
 
 def test_empty_sequences_and_alias(cuda_lib):
@@ -301,15 +463,21 @@ def test_packed_order_many_sequences(cuda_lib, n_seq, dtype, dk):
 
 def test_schedule_is_the_one_forced(cuda_lib, schedule):
     """The forced schedules are the ones launched; the automatic choice takes
-    the pair while every unit gets one in a wave, one CTA per unit beyond."""
+    a pair while every unit gets one in a wave (the WY-form pair for FP8
+    tiles), one CTA per unit beyond."""
     pick = cuda_lib.gdn_prefill_schedule
     if schedule == "pair":
         assert pick(4, 16, 128, 128) == "tc_cta_pair"
+        assert pick(4, 16, 128, 128, qdq="int8_g32") == "tc_cta_pair"
+    elif schedule == "wy":
+        assert pick(4, 16, 128, 128) == "tc_wy_pair"
+        assert pick(64, 16, 128, 128) == "tc_wy_pair"
+        assert pick(4, 16, 128, 128, qdq="int8_g32") == "tc_cta_pair"
     elif schedule == "single":
         assert pick(4, 16, 128, 128) == "tc_one_cta"
     else:
         assert pick(4, 16, 128, 128) == "tc_cta_pair"
+        assert pick(4, 16, 128, 128, qdq="none") == "tc_cta_pair"
         assert pick(64, 16, 128, 128) == "tc_one_cta"
     assert pick(4, 16, 128, 128, dtype=torch.float32) == "cuda_cores"
-    assert pick(4, 16, 128, 128, gate="per_key") == "cuda_cores"
-
+    assert pick(4, 16, 128, 128, gate="per_key", qdq="int8_g32") == "cuda_cores"

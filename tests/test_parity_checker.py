@@ -122,3 +122,38 @@ def test_relative_errors():
     x[1, 1] = 1.1                                   # unit 1 off by 10 %, unit 0 exact
     assert per_unit_rel_err(x, ref, axes=(1,)) == pytest.approx(0.1)
     assert rel_err(np.zeros(2), np.zeros(2)) == 0.0
+
+
+def test_element_guard_catches_one_corrupted_element_the_norm_misses():
+    """One element of a 4096 x 128 bf16-sized output off by 20 % of its row's
+    largest value moves the norm-wise error by about 2e-4 (under the 2e-3
+    bar) but fails the element-level guard; bf16 rounding of every element
+    (at most 2^-8 of the row's largest value) passes both."""
+    from parity import TOL, assert_rows_close
+    rng = np.random.default_rng(5)
+    ref = rng.standard_normal((4096, 128))
+    x = ref.astype(np.float32).astype(np.float64)
+    # round to bf16 (8-bit significands, nearest even) through the bit pattern
+    b = ref.astype(np.float32).view(np.uint32)
+    b = ((b + 0x7FFF + ((b >> 16) & 1)) & 0xFFFF0000).astype(np.uint32)
+    x = b.view(np.float32).astype(np.float64)
+    assert rel_err(x, ref) <= TOL["bf16"]
+    assert assert_rows_close(x, ref, "bf16") <= 2.0 ** -8
+    bad = x.copy()
+    bad[1234, 17] += 0.2 * np.abs(ref[1234]).max()
+    assert rel_err(bad, ref) <= TOL["bf16"]
+    with pytest.raises(AssertionError):
+        assert_rows_close(bad, ref, "bf16")
+
+
+def test_element_guard_on_rows_of_zeros():
+    """A row whose reference is zero is measured against 1e-6 of the tensor's
+    largest magnitude: a stray value there fails, an exact zero passes."""
+    from parity import assert_rows_close
+    ref = np.zeros((3, 8))
+    ref[0] = 1.0
+    x = ref.copy()
+    assert assert_rows_close(x, ref, "f32") == 0.0
+    x[2, 3] = 1e-3
+    with pytest.raises(AssertionError):
+        assert_rows_close(x, ref, "f32")
