@@ -239,8 +239,10 @@ __device__ __forceinline__ uint32_t fp8_codes(float x0, float x1, const ScaleRec
 
 // code pair (fp16) * c -> two fp32 values.
 __device__ __forceinline__ void dequant2(uint32_t code, float c, float &y0, float &y1) {
-  const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&code));
-  f2_unpack(f2_mul(f2_pack(f.x, f.y), f2_pack(c, c)), y0, y1);
+  float a, b;
+  h2_to_f32(code, a, b);
+  y0 = a * c;
+  y1 = b * c;
 }
 
 __device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t (&v)[32]) {
@@ -493,6 +495,12 @@ prefill_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       sm100::fence_proxy_async();
       sm100::tc_fence_before();
       __syncthreads();
+      // the hand-off leaves in three pieces as they are ready (Aqk now, T
+      // diag(beta) after the solve, W last), all counted on the chain's
+      // receive barrier of this slot
+      if (tid == 0 && !sm->abort)
+        sm100::bulk_copy_to_cluster(rx_buf_remote[b] + H_AQK, stg + H_AQK, kRxBytes - H_AQK,
+                                    rx_full_remote[b]);
       // the next chunk's MMA 1 runs during this chunk's solve (D1 has been read)
       if (warp == 4 && j + 1 < n_chunks) {
         const int nbuf = (j + 1) & 1;
@@ -554,39 +562,46 @@ prefill_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           }
           *reinterpret_cast<float4 *>(sT + (r0 + rr) * LDT + c0b + cc) = make_float4(-q.x, -q.y, -q.z, -q.w);
         }
-        asm volatile("bar.sync 3, 128;" ::: "memory");
-        // level 2: the lower-left 32x32 block: T_21 = -T_22 (A_21 T_11)
-        {
-          const int rr = tid >> 2, cc = (tid & 3) * 8;
-          const float *arow = sA + (32 + rr) * LDT;
-          const float *tcol = sT + cc;
-          float p[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      }
+      __syncthreads();
+      // level 2 (all 256 threads): the lower-left 32x32 block,
+      // T_21 = -T_22 (A_21 T_11); thread: row rr, columns cc .. cc + 3
+      {
+        const int rr = tid >> 3, cc = (tid & 7) * 4;
+        float a[32];  // the thread's row of A_21, then of T_22
 #pragma unroll
-          for (int m = 0; m < 32; ++m) {
-            const float a = arow[m];
-            const float4 t0v = *reinterpret_cast<const float4 *>(tcol + m * LDT);
-            const float4 t1v = *reinterpret_cast<const float4 *>(tcol + m * LDT + 4);
-            p[0] += a * t0v.x; p[1] += a * t0v.y; p[2] += a * t0v.z; p[3] += a * t0v.w;
-            p[4] += a * t1v.x; p[5] += a * t1v.y; p[6] += a * t1v.z; p[7] += a * t1v.w;
-          }
-          *reinterpret_cast<float4 *>(sP + rr * LDT + cc) = make_float4(p[0], p[1], p[2], p[3]);
-          *reinterpret_cast<float4 *>(sP + rr * LDT + cc + 4) = make_float4(p[4], p[5], p[6], p[7]);
-          asm volatile("bar.sync 3, 128;" ::: "memory");
-          const float *trow = sT + (32 + rr) * LDT + 32;
-          const float *pcol = sP + cc;
-          float q[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-          for (int m = 0; m < 32; ++m) {
-            const float t = trow[m];
-            const float4 p0v = *reinterpret_cast<const float4 *>(pcol + m * LDT);
-            const float4 p1v = *reinterpret_cast<const float4 *>(pcol + m * LDT + 4);
-            q[0] += t * p0v.x; q[1] += t * p0v.y; q[2] += t * p0v.z; q[3] += t * p0v.w;
-            q[4] += t * p1v.x; q[5] += t * p1v.y; q[6] += t * p1v.z; q[7] += t * p1v.w;
-          }
-          float *tout = sT + (32 + rr) * LDT + cc;
-          *reinterpret_cast<float4 *>(tout) = make_float4(-q[0], -q[1], -q[2], -q[3]);
-          *reinterpret_cast<float4 *>(tout + 4) = make_float4(-q[4], -q[5], -q[6], -q[7]);
+        for (int m = 0; m < 32; m += 4) {
+          const float4 a4 = *reinterpret_cast<const float4 *>(sA + (32 + rr) * LDT + m);
+          a[m] = a4.x; a[m + 1] = a4.y; a[m + 2] = a4.z; a[m + 3] = a4.w;
         }
+        const float *tcol = sT + cc;
+        float4 p = make_float4(0.f, 0.f, 0.f, 0.f), p2 = p;
+#pragma unroll
+        for (int m = 0; m < 32; m += 2) {
+          const float4 t4 = *reinterpret_cast<const float4 *>(tcol + m * LDT);
+          const float4 u4 = *reinterpret_cast<const float4 *>(tcol + (m + 1) * LDT);
+          p.x += a[m] * t4.x; p.y += a[m] * t4.y; p.z += a[m] * t4.z; p.w += a[m] * t4.w;
+          p2.x += a[m + 1] * u4.x; p2.y += a[m + 1] * u4.y; p2.z += a[m + 1] * u4.z; p2.w += a[m + 1] * u4.w;
+        }
+        *reinterpret_cast<float4 *>(sP + rr * LDT + cc) =
+            make_float4(p.x + p2.x, p.y + p2.y, p.z + p2.z, p.w + p2.w);
+#pragma unroll
+        for (int m = 0; m < 32; m += 4) {
+          const float4 a4 = *reinterpret_cast<const float4 *>(sT + (32 + rr) * LDT + 32 + m);
+          a[m] = a4.x; a[m + 1] = a4.y; a[m + 2] = a4.z; a[m + 3] = a4.w;
+        }
+        __syncthreads();
+        const float *pcol = sP + cc;
+        float4 q = make_float4(0.f, 0.f, 0.f, 0.f), q2 = q;
+#pragma unroll
+        for (int m = 0; m < 32; m += 2) {
+          const float4 p4 = *reinterpret_cast<const float4 *>(pcol + m * LDT);
+          const float4 v4 = *reinterpret_cast<const float4 *>(pcol + (m + 1) * LDT);
+          q.x += a[m] * p4.x; q.y += a[m] * p4.y; q.z += a[m] * p4.z; q.w += a[m] * p4.w;
+          q2.x += a[m + 1] * v4.x; q2.y += a[m + 1] * v4.y; q2.z += a[m + 1] * v4.z; q2.w += a[m + 1] * v4.w;
+        }
+        *reinterpret_cast<float4 *>(sT + (32 + rr) * LDT + cc) =
+            make_float4(-(q.x + q2.x), -(q.y + q2.y), -(q.z + q2.z), -(q.w + q2.w));
       }
       __syncthreads();
       // ---- T diag(beta gamma) -> hi/lo (B of the W product, in the W area)
@@ -628,6 +643,9 @@ prefill_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       sm100::fence_proxy_async();
       sm100::tc_fence_before();
       __syncthreads();
+      if (tid == 0 && !sm->abort)
+        sm100::bulk_copy_to_cluster(rx_buf_remote[b] + H_THI, stg + H_THI, H_AQK - H_THI,
+                                    rx_full_remote[b]);
       // ---- W^T [k][t hi part | t lo part] = K^T (T diag(beta gamma))^T ----
       if (warp == 0) {
         sm100::tc_fence_after();
@@ -659,7 +677,8 @@ prefill_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       sm100::tc_fence_before();
       __syncthreads();
       if (tid == 0 && !sm->abort)
-        sm100::bulk_copy_to_cluster(rx_buf_remote[b], stg, kRxBytes, rx_full_remote[b]);
+        sm100::bulk_copy_to_cluster(rx_buf_remote[b] + H_WHI, stg + H_WHI, H_THI - H_WHI,
+                                    rx_full_remote[b]);
     }
     // an aborted producer lets its TMA loads land before leaving
     if (tid == 0 && sm->abort) {
@@ -782,18 +801,18 @@ prefill_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         sm100::tc_fence_after();
         if (got && sm100::elect_one()) {
           if (!u_done) issue_u(it);
-#pragma unroll
+#pragma unroll 1
           for (int ks = 0; ks < 8; ++ks)
             sm100::mma_f16_ts(tmem + TM_X, tmem + TM_S0C + 8u * ks,
                               mndesc(rx + H_WHI + (uint32_t)ks * 2048u, 16384), ID_X, ks > 0);
           if (!exact) {
-#pragma unroll
+#pragma unroll 1
             for (int ks = 0; ks < 8; ++ks)
               sm100::mma_f16_ts(tmem + TM_X, tmem + TM_O2 + 8u * ks,
                                 mndesc(rx + H_WHI + (uint32_t)ks * 2048u, 16384), ID_X64, 1);
           }
           sm100::mma_commit(&sm->bar_x);
-#pragma unroll
+#pragma unroll 1
           for (int ks = 0; ks < 8; ++ks)
             sm100::mma_f16_ts(tmem + TM_O1, tmem + TM_S0C + 8u * ks,
                               kdesc(kq + 8192u + (uint32_t)(ks >> 2) * 16384u + (uint32_t)(ks & 3) * 32u),
@@ -910,16 +929,32 @@ prefill_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       {
         wait_local(&sm->bar_o2, (uint32_t)(it & 1), sm, err);
         sm100::tc_fence_after();
+        if (tid == 0 && !sm->abort) {
+          // the receive slot has been read (W by X, T diag(beta) by U, Aqk by
+          // O part 2; this thread has seen those MMAs complete): arm it for
+          // chunk it + 2, then hand it back to the producer
+          if (it + 2 < n_chunks) {
+            sm100::mbar_arrive_expect_tx(&sm->rx_full[kb], kRxBytes);
+            sm->rx_pend[kb] = 1 + (((it + 2) >> 1) & 1);
+          }
+          sm100::mbar_arrive_cluster_relaxed(rx_free_remote[kb]);
+        }
         float o1[32], o2[32];
         sm100::tmem_ld32(tmem + lane_off + TM_O1 + 32 * wg, o1);
         sm100::tmem_ld32(tmem + lane_off + TM_O2 + 32 * wg, o2);
         const int cnt = n - 32 * wg;
-        __nv_bfloat16 *dst = o + ((tb + 32 * wg) * H + h) * kD + row;
+        unsigned short *dst =
+            reinterpret_cast<unsigned short *>(o + ((tb + 32 * wg) * H + h) * kD + row);
         const long long ts = (long long)H * kD;
         const float ss = scale * s0;
 #pragma unroll
-        for (int t = 0; t < 32; ++t)
-          if (t < cnt) dst[t * ts] = __float2bfloat16_rn(fmaf(ss, o1[t], scale * o2[t]));
+        for (int t = 0; t < 32; t += 2) {
+          const __nv_bfloat162 p2 =
+              __floats2bfloat162_rn(fmaf(ss, o1[t], scale * o2[t]), fmaf(ss, o1[t + 1], scale * o2[t + 1]));
+          const uint32_t w = *reinterpret_cast<const uint32_t *>(&p2);
+          if (t < cnt) dst[t * ts] = (unsigned short)(w & 0xffffu);
+          if (t + 1 < cnt) dst[(t + 1) * ts] = (unsigned short)(w >> 16);
+        }
       }
       if (warp == 7 && it + 2 < n_chunks)
         finish_chain_gates(&sm->gt[(it + 2) % 3], graw, chunk_len(it + 2), lane);
@@ -929,15 +964,6 @@ prefill_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       // ---- (F) the QDQ ----
       wait_local(&sm->bar_m5, (uint32_t)(it & 1), sm, err);
       sm100::tc_fence_after();
-      if (tid == 0 && !sm->abort) {
-        // this receive slot has been read (W by X, T diag(beta) by U, Aqk by
-        // O part 2): arm it for chunk it + 2, then release it to the producer
-        if (it + 2 < n_chunks) {
-          sm100::mbar_arrive_expect_tx(&sm->rx_full[kb], kRxBytes);
-          sm->rx_pend[kb] = 1 + (((it + 2) >> 1) & 1);
-        }
-        sm100::mbar_arrive_cluster(rx_free_remote[kb]);
-      }
       // the S update has read K: the buffer takes chunk it + 2
       if (tid == 224 && it + 2 < n_chunks && !sm->abort) issue_qk(it + 2);
       {
@@ -946,7 +972,9 @@ prefill_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         sm100::tmem_ld32(tmem + lane_off + TM_S + 64 * wg + 32, *reinterpret_cast<float(*)[32]>(y + 32));
         float mh = 0.f;
 #pragma unroll
-        for (int i = 0; i < 64; ++i) mh = fmaxf(mh, fabsf(y[i]));
+        for (int i = 0; i < 64; i += 2) {
+          asm("max.f32 %0, %1, %2, %3;" : "=f"(mh) : "f"(mh), "f"(fabsf(y[i])), "f"(fabsf(y[i + 1])));
+        }
         mh = group_max<32>(mh);
         // one FP8 tile = value columns 64 tile .. + 63 = warps (2 tile, 2 tile + 1)
         // of both warpgroups

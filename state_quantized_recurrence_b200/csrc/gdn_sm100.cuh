@@ -58,6 +58,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of a phase (no suspension).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 __device__ __forceinline__ uint64_t global_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -65,11 +78,10 @@ __device__ __forceinline__ uint64_t global_ns() {
 }
 
 // Bounded wait: true once the phase with `parity` completed, false when
-// `limit_ns` nanoseconds passed first (a limit of 0 gives up as soon as one
-// test finds the phase incomplete).
+// `limit_ns` nanoseconds passed first (a limit of 0: one non-blocking test).
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
+  if (limit_ns == 0) return mbar_test_wait(bar, parity);
   if (mbar_try_wait(bar, parity)) return true;
-  if (limit_ns == 0) return false;
   const uint64_t start = global_ns();
   for (;;) {
 #pragma unroll 1
@@ -97,6 +109,15 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t remote_bar) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar)
                : "memory");
 }
+// The same without release ordering: for a signal whose only meaning is that
+// asynchronous (tensor-core) reads this thread has already seen complete
+// are done, so that no prior write of this thread needs to be made visible
+// first (a release would also wait for the thread's outstanding global
+// stores).
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t remote_bar) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar)
+               : "memory");
+}
 // Phase test with cluster-scope acquire (the phase may be completed by another
 // CTA's arrival or by a bulk copy from another CTA), with the short suspend
 // hint of mbar_try_wait.
@@ -111,9 +132,20 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t pa
       : "memory");
   return ok != 0;
 }
+__device__ __forceinline__ bool mbar_test_wait_cluster(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
+  if (limit_ns == 0) return mbar_test_wait_cluster(bar, parity);
   if (mbar_try_wait_cluster(bar, parity)) return true;
-  if (limit_ns == 0) return false;
   const uint64_t start = global_ns();
   for (;;) {
 #pragma unroll 1

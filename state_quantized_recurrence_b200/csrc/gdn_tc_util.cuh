@@ -26,12 +26,32 @@ __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
   return *reinterpret_cast<uint32_t *>(&h);
 }
 
-// hi = fp16(x), lo = fp16(x - hi), packed in pairs.
+// x - (the low / high fp16 of an fp16 pair), exactly, as one mixed-precision
+// FMA (fp16 operands, fp32 addend and result) on the FMA pipe instead of a
+// conversion.
+__device__ __forceinline__ float sub_h_lo(float x, uint32_t h2) {
+  float d;
+  asm("{\n\t.reg .f16 l, h, m;\n\tmov.b32 {l, h}, %1;\n\tmov.b16 m, 0xBC00;\n\t"
+      "fma.rn.f32.f16 %0, l, m, %2;\n\t}" : "=f"(d) : "r"(h2), "f"(x));
+  return d;
+}
+__device__ __forceinline__ float sub_h_hi(float x, uint32_t h2) {
+  float d;
+  asm("{\n\t.reg .f16 l, h, m;\n\tmov.b32 {l, h}, %1;\n\tmov.b16 m, 0xBC00;\n\t"
+      "fma.rn.f32.f16 %0, h, m, %2;\n\t}" : "=f"(d) : "r"(h2), "f"(x));
+  return d;
+}
+// The two fp32 values of an fp16 pair (exact): mixed-precision adds of -0.
+__device__ __forceinline__ void h2_to_f32(uint32_t h2, float &a, float &b) {
+  asm("{\n\t.reg .f16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "add.rn.f32.f16 %0, l, 0f80000000;\n\tadd.rn.f32.f16 %1, h, 0f80000000;\n\t}"
+      : "=f"(a), "=f"(b) : "r"(h2));
+}
+
+// hi = fp16(x), lo = fp16(x - hi), packed in pairs (x - hi is exact in fp32).
 __device__ __forceinline__ void split_h2(float a, float b, uint32_t &hi, uint32_t &lo) {
-  __half2 h = __floats2half2_rn(a, b);
-  float2 hf = __half22float2(h);
-  hi = *reinterpret_cast<uint32_t *>(&h);
-  lo = pack_h2(a - hf.x, b - hf.y);
+  hi = pack_h2(a, b);
+  lo = pack_h2(sub_h_lo(a, hi), sub_h_hi(b, hi));
 }
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
