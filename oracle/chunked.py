@@ -20,13 +20,35 @@ the default) and the WY decomposition of the delta rule:
 
 and the state QDQ at the chunk end.  Equality with the token recurrence (QDQ
 off) is the pin of this algebra.
+
+Optionally (``w_qdq="fp8_row"``) the WY-transformed W itself is fake-quantized
+before it is used, the pages' second, independent QDQ site (PR #2497 "GDN
+state/W QAT foundation", What and Usage sections: dynamic FP8 E4M3 on W, the
+quantizer keeping the batch, token and head axes): one scale per row of W
+(per token and head), amax over the key axis, scale = amax / 448 with a
+zero guard, all in fp32 like the state codec (:func:`w_row_qdq`).
 """
 
 from __future__ import annotations
 
 import numpy as np
 
-from . import CHUNK, _f64, dense_cu_seqlens, qdq as _qdq
+from . import CHUNK, _f64, dense_cu_seqlens, e4m3 as _e4m3, qdq as _qdq
+
+
+def w_row_qdq(W):
+    """Dynamic FP8 E4M3 QDQ of W [n, d_k], one scale per row: in fp32,
+    s = amax / 448 over the row (IEEE division), code = E4M3(fl32(w / s))
+    (nearest, ties to even, saturating), y = fl32(code * s); an all-zero row
+    stays zero.  Returns (y, codes, scales [n, 1]) as fp32."""
+    Wf = np.asarray(W, dtype=np.float32)
+    amax = np.abs(Wf).max(axis=-1, keepdims=True)
+    s = (amax / np.float32(448.0)).astype(np.float32)
+    safe = np.where(s > 0, s, np.float32(1.0)).astype(np.float32)
+    codes = _e4m3((Wf / safe).astype(np.float32))
+    y = (codes * safe).astype(np.float32)
+    y = np.where(amax > 0, y, np.float32(0.0)).astype(np.float32)
+    return y, codes, s
 
 
 def forward_substitution(A: np.ndarray) -> np.ndarray:
@@ -55,7 +77,7 @@ def neumann_inverse(A: np.ndarray, degree: int) -> np.ndarray:
 
 
 def chunk_step(Q, K, V, g, beta, H0, *, per_key_gate: bool, scale: float,
-               solve="exact"):
+               solve="exact", w_qdq: str = "none"):
     """One chunk: returns (O [n, d_v], H_n [d_k, d_v]) in fp64."""
     n = K.shape[0]
     if per_key_gate:
@@ -72,6 +94,8 @@ def chunk_step(Q, K, V, g, beta, H0, *, per_key_gate: bool, scale: float,
     else:
         T = neumann_inverse(A, int(solve[1]))
     W = T @ (beta[:, None] * (K * gamma))
+    if w_qdq == "fp8_row":
+        W = w_row_qdq(W)[0].astype(np.float64)
     U = T @ (beta[:, None] * V)
     V_new = U - W @ H0
     Aqk = np.tril(np.einsum("rc,ic,ric->ri", Q, K, D))
@@ -82,7 +106,8 @@ def chunk_step(Q, K, V, g, beta, H0, *, per_key_gate: bool, scale: float,
 
 
 def chunked_wy(q, k, v, g, beta, state_in, cu_seqlens, *, per_key_gate: bool,
-               qdq: str = "none", chunk: int = CHUNK, solve="exact"):
+               qdq: str = "none", chunk: int = CHUNK, solve="exact",
+               w_qdq: str = "none"):
     """Chunked prefix over packed sequences (same layout as
     :func:`oracle.recurrence`).  QDQ (if any) runs after every chunk."""
     q, k, v, g, beta = (_f64(x) for x in (q, k, v, g, beta))
@@ -108,7 +133,7 @@ def chunked_wy(q, k, v, g, beta, state_in, cu_seqlens, *, per_key_gate: bool,
                 O, Hs = chunk_step(q[c0:c1, h], k[c0:c1, h], v[c0:c1, h],
                                    g[c0:c1, h], beta[c0:c1, h], Hs,
                                    per_key_gate=per_key_gate, scale=scale,
-                                   solve=solve)
+                                   solve=solve, w_qdq=w_qdq)
                 o[c0:c1, h] = O
                 if qdq != "none":
                     Hs = _qdq(Hs.astype(np.float32), qdq)[0].astype(np.float64)

@@ -88,6 +88,14 @@ PY_MUTANTS = [
     ("carry without state decay", "Hn = gamma[n - 1][:, None] * H0 +", "Hn = H0 +"),
     ("substitution sign", "T[r, :] -= A[r, i] * T[i, :]", "T[r, :] += A[r, i] * T[i, :]"),
     ("substitution transposed", "T[r, :] -= A[r, i] * T[i, :]", "T[r, :] -= A[i, r] * T[i, :]"),
+    ("W QDQ per column", "amax = np.abs(Wf).max(axis=-1, keepdims=True)",
+     "amax = np.abs(Wf).max(axis=0, keepdims=True)"),
+    ("W QDQ scale constant", "s = (amax / np.float32(448.0)).astype(np.float32)",
+     "s = (amax / np.float32(240.0)).astype(np.float32)"),
+    ("W QDQ on U instead of W", "    U = T @ (beta[:, None] * V)\n",
+     "    U = T @ (beta[:, None] * V)\n    if w_qdq == \"fp8_row\":\n        U = w_row_qdq(U)[0].astype(np.float64)\n"),
+    ("W QDQ without the zero guard",
+     "safe = np.where(s > 0, s, np.float32(1.0)).astype(np.float32)", "safe = s"),
     ("Neumann sign", "P = -A @ P", "P = A @ P"),
     ("Neumann one term short", "for _ in range(degree):", "for _ in range(degree - 1):"),
 ]
@@ -155,6 +163,10 @@ PINS = [
     ("qdq placement int8", lambda: rec.test_qdq_placement_prefill("int8_g32")),
     ("qdq placement fp8", lambda: rec.test_qdq_placement_prefill("fp8_tile64")),
     ("qdq placement decode", rec.test_qdq_placement_decode),
+    ("w qdq grid and row scale", rec.test_w_row_qdq_grid_and_per_row_scale),
+    ("w qdq = tile codec per row", rec.test_w_row_qdq_matches_the_tile_codec_row_by_row),
+    ("w qdq beta 0", rec.test_w_qdq_leaves_beta_zero_chunks_alone),
+    ("w qdq one-hot keys", rec.test_w_qdq_on_one_hot_keys_is_the_identity_within_an_ulp),
 ]
 
 

@@ -281,3 +281,85 @@ def test_generator_inputs_run_tiny():
     rebuilt = (codes.reshape(1, 2, 64, 2, 32) *
                scales.reshape(1, 2, 64, 2, 1)).reshape(s.shape).astype(np.float32)
     np.testing.assert_array_equal(s.astype(np.float32), rebuilt)
+
+
+# ---------------------------------------------------------------- W QDQ ----
+# The optional FP8 QDQ of the WY-transformed W (one dynamic scale per row of
+# W, i.e. per token and head, over the key axis; PR #2497 "GDN state/W QAT
+# foundation", What and Usage sections).
+
+def _w_rows(seed=3):
+    rng = np.random.default_rng(seed)
+    W = rng.standard_normal((64, 128)) * np.exp2(rng.integers(-30, 20, (64, 1)))
+    W[5] = 0.0                      # an all-zero row
+    W[9] = 0.0
+    W[9, 17] = -3.25                # a row with one nonzero element
+    return W.astype(np.float32)
+
+
+def test_w_row_qdq_grid_and_per_row_scale():
+    """Every value is code * s_row with code on the E4M3 grid; the row's
+    largest magnitude maps to exactly +-448 (so the scale is the row's own,
+    not a column's or the tensor's); a zero row stays zero; idempotent."""
+    import torch
+    from test_oracle_codecs import e4m3_value_set
+    W = _w_rows()
+    y, codes, s = chunked.w_row_qdq(W)
+    grid = e4m3_value_set()
+    assert set(np.unique(codes).astype(np.float64)) <= grid
+    nz = np.abs(W).max(axis=1) > 0
+    np.testing.assert_array_equal(np.abs(codes[nz]).max(axis=1), 448.0)
+    assert not y[~nz].any() and not codes[~nz].any()
+    np.testing.assert_array_equal(y[nz], (codes[nz] * s[nz]).astype(np.float32))
+    # the code rounding against the library's float8 cast of the same quotients
+    q = (W[nz] / s[nz]).astype(np.float32)
+    lib = torch.from_numpy(q).to(torch.float8_e4m3fn).float().numpy()
+    np.testing.assert_array_equal(codes[nz], lib)
+    y2 = chunked.w_row_qdq(y)[0]
+    np.testing.assert_array_equal(y2, y)
+
+
+def test_w_row_qdq_matches_the_tile_codec_row_by_row():
+    """Each row on its own in column 0 of an otherwise zero [128 x 64] FP8
+    tile goes through the C state codec (an independent implementation of
+    the same scale and rounding) to the same values."""
+    W = _w_rows(4)
+    y = chunked.w_row_qdq(W)[0]
+    tiles = np.zeros((W.shape[0], 128, 64), np.float32)
+    tiles[:, :, 0] = W
+    ref = oracle.qdq(tiles, "fp8_tile64")[0][:, :, 0]
+    np.testing.assert_array_equal(y, ref)
+
+
+def test_w_qdq_leaves_beta_zero_chunks_alone():
+    """beta = 0 makes W = 0 (zero rows): the W QDQ changes nothing."""
+    case = gs.Case("wq0", n_seq=1, H=2, d_k=64, d_v=64, T=100, dtype="f32",
+                   qdq="fp8_tile64", state="normal", seed=131)
+    inp = gs.generate(case)
+    inp["beta"] = np.zeros_like(inp["beta"])
+    a = chunked.chunked_dense(inp, case, qdq="fp8_tile64")
+    b = chunked.chunked_dense(inp, case, qdq="fp8_tile64", w_qdq="fp8_row")
+    np.testing.assert_array_equal(a[0], b[0])
+    np.testing.assert_array_equal(a[1], b[1])
+
+
+def test_w_qdq_on_one_hot_keys_is_the_identity_within_an_ulp():
+    """Mutually orthogonal one-hot keys give A = 0, T = I and W rows
+    beta_t gamma_t e_t: a one-element row keeps its value up to the fp32
+    rounding of its scale, so the chunk's result moves by at most a few
+    ulp - whereas a QDQ applied to U, V or K (dense rows) moves it by the
+    FP8 step."""
+    import torch
+    n, d = 40, 64
+    q = torch.randn((1, n, 1, d), generator=torch.Generator().manual_seed(5))
+    k = torch.zeros((1, n, 1, d))
+    k[0, np.arange(n), 0, np.arange(n)] = 1.0
+    v = torch.randn((1, n, 1, d), generator=torch.Generator().manual_seed(6))
+    g = torch.full((1, n, 1), -0.05)
+    beta = torch.full((1, n, 1), 0.7)
+    st = torch.randn((1, 1, d, d), generator=torch.Generator().manual_seed(7)) * 0.1
+    cu = np.array([0, n])
+    a = chunked.chunked_wy(q, k, v, g, beta, st, cu, per_key_gate=False)
+    b = chunked.chunked_wy(q, k, v, g, beta, st, cu, per_key_gate=False, w_qdq="fp8_row")
+    assert np.abs(b[0] - a[0]).max() <= 1e-6 * np.abs(a[0]).max()
+    assert np.abs(b[1] - a[1]).max() <= 1e-6 * np.abs(a[1]).max()
