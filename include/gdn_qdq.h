@@ -266,6 +266,37 @@ gdn_status gdn_prefill_backward_static(const void *q, const void *k, const void 
                                        float *dbeta, float *dstate_in, void *cuda_stream);
 
 /*
+ * gdn_prefill_w_qdq - gdn_prefill with the second, independent QDQ site of
+ * the pages: dynamic FP8 E4M3 fake quantization of the WY-transformed W
+ * activations (PR #2497 "GDN state/W QAT foundation", What section: "independent
+ * dynamic FP8 fake QDQ to WY-transformed W activations"; Usage section: the W
+ * quantizer keeps axes (0, 1, 2), i.e. batch, token and head).
+ *
+ * In every 64-token chunk, W = T diag(beta gamma) K ([chunk tokens, d_k])
+ * is replaced by its QDQ before V_new = U - W H0 is formed: one scale per
+ * row of W (one token of one head), s = amax over the d_k keys / 448 in
+ * fp32, with a zero guard; code = E4M3(x / s) rounded to nearest even and
+ * saturated at +-448; value = code * s.  Everything else is gdn_prefill.
+ *
+ * w_qdq = GDN_W_QDQ_NONE is exactly gdn_prefill.  GDN_W_QDQ_FP8_E4M3_ROW is
+ * supported for bf16 q/k/v, scalar (GDN) gates, d_k = d_v = 128 and
+ * qdq = GDN_QDQ_FP8_E4M3_TILE64, and always runs the WY-form CTA pair
+ * kernel; other combinations return GDN_ERR_UNSUPPORTED before any launch.
+ * Arguments, layouts, ownership and errors as for gdn_prefill.
+ */
+typedef enum {
+    GDN_W_QDQ_NONE = 0,
+    GDN_W_QDQ_FP8_E4M3_ROW = 1   /* one scale per row of W (token, head) */
+} gdn_w_qdq_mode;
+gdn_status gdn_prefill_w_qdq(const void *q, const void *k, const void *v,
+                             const float *g, const float *beta,
+                             const float *state_in, const int32_t *cu_seqlens,
+                             int n_seq, int T, int H, int d_k, int d_v,
+                             gdn_dtype dt, gdn_gate_kind gk, gdn_qdq_mode qdq,
+                             gdn_w_qdq_mode w_qdq, void *o, float *state_out,
+                             void *cuda_stream);
+
+/*
  * gdn_prefill_schedule - which prefill kernel gdn_prefill launches for these
  * shapes and this codec on the current device, under the current
  * GDN_PREFILL_CTA_PAIR and GDN_PREFILL_WY settings (the same selection code).

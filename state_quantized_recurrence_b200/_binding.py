@@ -14,6 +14,7 @@ library_path = os.path.join(_PKG, "libgdn_qdq.so")
 GDN_STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED",
               3: "GDN_ERR_CUDA", 4: "GDN_ERR_TIMEOUT"}
 GDN_QDQ = {"none": 0, "fp8_tile64": 1, "int8_g32": 2, "int8_g16": 3, "int8_g64": 4}
+GDN_W_QDQ = {"none": 0, "fp8_row": 1}
 GDN_DTYPE = {torch.bfloat16: 0, torch.float32: 1}
 GDN_GATE = {"scalar": 0, "per_key": 1}
 
@@ -35,6 +36,8 @@ def _load() -> ctypes.CDLL:
     L.gdn_prefill.restype = I
     L.gdn_prefill_neumann.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, P, P, P]
     L.gdn_prefill_neumann.restype = I
+    L.gdn_prefill_w_qdq.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, P, P, P]
+    L.gdn_prefill_w_qdq.restype = I
     L.gdn_prefill_backward_workspace_bytes.argtypes = [I, I, I, I, I, I]
     L.gdn_prefill_backward_workspace_bytes.restype = ctypes.c_size_t
     L.gdn_prefill_backward.argtypes = ([P] * 7 + [I] * 8 + [P, P, P, ctypes.c_size_t]
@@ -133,15 +136,19 @@ def _gate_kind(g: torch.Tensor, lead: int) -> str:
 
 def gdn_prefill_into(q, k, v, g, beta, state_in, cu_seqlens, o, state_out,
                      qdq: str = "fp8_tile64", stream=None,
-                     neumann_degree: Optional[int] = None) -> None:
+                     neumann_degree: Optional[int] = None, w_qdq: str = "none") -> None:
     """Chunked prefix writing into preallocated ``o`` and ``state_out``.
 
     Dense: q, k [B, T, H, d_k], v/o [B, T, H, d_v]; packed (cu_seqlens int32
     [n_seq + 1]): [1, T_total, H, d].  g: fp32 [.., H] or [.., H, d_k];
     beta fp32 [.., H]; states fp32 [n_seq, H, d_k, d_v].  ``neumann_degree``
     (1, 3, 7, 15, 31 or 63) selects the approximate solve
-    (gdn_prefill_neumann); None the exact one.
+    (gdn_prefill_neumann); None the exact one.  ``w_qdq="fp8_row"`` adds the
+    FP8 QDQ of the WY-transformed W, one scale per row (gdn_prefill_w_qdq).
     """
+    _need(w_qdq in GDN_W_QDQ, "w_qdq must be 'none' or 'fp8_row'")
+    _need(w_qdq == "none" or neumann_degree is None,
+          "the W codec is not offered with the Neumann solve")
     dev = _check_dev(q, k, v, g, beta, state_in, cu_seqlens, o, state_out)
     _need(q.dim() == 4 and k.shape == q.shape and v.dim() == 4, "q, k, v must be [B, T, H, d]")
     B, T, H, d_k = q.shape
@@ -168,7 +175,9 @@ def gdn_prefill_into(q, k, v, g, beta, state_in, cu_seqlens, o, state_out,
             n_seq, T_arg, H, d_k, d_v, GDN_DTYPE[q.dtype], GDN_GATE[gk], GDN_QDQ[qdq])
     with torch.cuda.device(dev):
         tail = (_ptr(o), _ptr(state_out), _stream(stream, dev))
-        if neumann_degree is None:
+        if w_qdq != "none":
+            s, where = lib.gdn_prefill_w_qdq(*args, GDN_W_QDQ[w_qdq], *tail), "gdn_prefill_w_qdq"
+        elif neumann_degree is None:
             s, where = lib.gdn_prefill(*args, *tail), "gdn_prefill"
         else:
             s, where = (lib.gdn_prefill_neumann(*args, int(neumann_degree), *tail),
@@ -269,7 +278,7 @@ def gdn_prefill_backward_static(q, k, v, g, beta, d_o, state_in=None, cu_seqlens
 
 
 def gdn_prefill(q, k, v, g, beta, state_in=None, cu_seqlens=None, qdq: str = "fp8_tile64",
-                stream=None, neumann_degree: Optional[int] = None):
+                stream=None, neumann_degree: Optional[int] = None, w_qdq: str = "none"):
     """Chunked prefix; returns ``(o, state_out)`` (allocated with torch).
     ``neumann_degree`` (1, 3, 7, 15, 31 or 63) replaces the exact triangular
     solve of every chunk by the truncated Neumann series of that degree
@@ -279,7 +288,7 @@ def gdn_prefill(q, k, v, g, beta, state_in=None, cu_seqlens=None, qdq: str = "fp
     state_out = torch.empty((n_seq, q.shape[2], q.shape[3], v.shape[3]), dtype=torch.float32,
                             device=q.device)
     gdn_prefill_into(q, k, v, g, beta, state_in, cu_seqlens, o, state_out, qdq, stream,
-                     neumann_degree)
+                     neumann_degree, w_qdq)
     return o, state_out
 
 

@@ -294,11 +294,12 @@ gdn_status launch_pair_one(const CUtensorMap &mq, const CUtensorMap &mk, const C
 
 // The WY-form pair (FP8 tiles): the producer CTA also forms W and hands it
 // over; the chain CTA keeps the state transposed in TMEM.
+template <bool WQ>
 gdn_status launch_wy_one(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv_sw,
                          const float *g, const float *beta, const float *state_in,
                          const int32_t *cu, int T, int H, float scale, __nv_bfloat16 *o,
                          float *state_out, unsigned *err, unsigned units, cudaStream_t st) {
-  auto kern = gdn::wy::prefill_wy_kernel;
+  auto kern = gdn::wy::prefill_wy_kernel<WQ>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)gdn::wy::kSmemBytes) != cudaSuccess)
     return GDN_ERR_CUDA;
@@ -366,7 +367,7 @@ bool tc_path(gdn_dtype dt, gdn_gate_kind gk, int d_k, int d_v) {
 gdn_status launch_prefill_tc(const void *q, const void *k, const void *v, const float *g,
                              const float *beta, const float *state_in, const int32_t *cu,
                              int n_seq, int T, int H, int kind, int group, void *o,
-                             float *state_out, unsigned *err, cudaStream_t st) {
+                             float *state_out, unsigned *err, cudaStream_t st, bool w_qdq) {
   const long long blocks = (long long)n_seq * H;
   if (blocks > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
   const long long rows = cu ? (long long)T : (long long)n_seq * T;
@@ -382,13 +383,16 @@ gdn_status launch_prefill_tc(const void *q, const void *k, const void *v, const 
   const unsigned nb = (unsigned)blocks;
   CUtensorMap mo;  // outputs [rows, H, 128] bf16, stored by whole 64-token chunks
   if ((s = make_token_map(&mo, o, H, rows, true)) != GDN_OK) return s;
-  if (use_pair(blocks)) {
+  if (w_qdq || use_pair(blocks)) {
     if (blocks > 0x3fffffffLL) return GDN_ERR_UNSUPPORTED;
-    if (use_wy(kind)) {
+    if (w_qdq || use_wy(kind)) {
       CUtensorMap mvs;  // V tiles 128B-swizzled: the A operand of U^T = V^T (T diag(beta))^T
       if ((s = make_token_map(&mvs, v, H, rows, true)) != GDN_OK) return s;
-      return launch_wy_one(mq, mk, mvs, g, beta, state_in, cu, T, H, scale, oo, state_out, err,
-                           nb, st);
+      if (w_qdq)
+        return launch_wy_one<true>(mq, mk, mvs, g, beta, state_in, cu, T, H, scale, oo, state_out,
+                                   err, nb, st);
+      return launch_wy_one<false>(mq, mk, mvs, g, beta, state_in, cu, T, H, scale, oo, state_out,
+                                  err, nb, st);
     }
 #define GDN_TP(QK, GR) \
   launch_pair_one<QK, GR>(mq, mk, mv, mo, g, beta, state_in, cu, T, H, scale, oo, state_out, err, nb, st)
@@ -462,13 +466,19 @@ gdn_status prefill_impl(const void *q, const void *k, const void *v, const float
                         const float *beta, const float *state_in, const int32_t *cu_seqlens,
                         int n_seq, int T, int H, int d_k, int d_v, gdn_dtype dt,
                         gdn_gate_kind gk, gdn_qdq_mode qdq, int neu_m, void *o,
-                        float *state_out, void *cuda_stream) {
+                        float *state_out, void *cuda_stream,
+                        gdn_w_qdq_mode w_qdq = GDN_W_QDQ_NONE) {
   if (T < 0) return GDN_ERR_INVALID_ARG;
   const long long rows = cu_seqlens ? (long long)T : (long long)n_seq * T;
   gdn_status s = check_common(q, k, v, g, beta, o, n_seq, H, d_k, d_v, dt, gk, qdq, rows);
   if (s != GDN_OK) return s;
   int kind = 0, group = 32;
   if (!qdq_params(qdq, d_v, &kind, &group)) return GDN_ERR_UNSUPPORTED;
+  if (w_qdq != GDN_W_QDQ_NONE && w_qdq != GDN_W_QDQ_FP8_E4M3_ROW) return GDN_ERR_UNSUPPORTED;
+  // the W codec is built on the WY-form pair: bf16 GDN at d = 128 with FP8 state tiles
+  if (w_qdq != GDN_W_QDQ_NONE &&
+      (neu_m != 0 || !tc_path(dt, gk, d_k, d_v) || kind != gdn::kQdqFp8Tile))
+    return GDN_ERR_UNSUPPORTED;
   if (n_seq == 0) return GDN_OK;
   if (!state_out || !aligned(state_out, 16)) return GDN_ERR_INVALID_ARG;
   if (state_in && !aligned(state_in, 16)) return GDN_ERR_INVALID_ARG;
@@ -483,7 +493,7 @@ gdn_status prefill_impl(const void *q, const void *k, const void *v, const float
   // CUDA-core kernel for every dtype.  Both compute the same chunked algebra.
   if (neu_m == 0 && tc_path(dt, gk, d_k, d_v))
     return launch_prefill_tc(q, k, v, g, beta, state_in, cu_seqlens, n_seq, T, H, kind, group, o,
-                             state_out, err, st);
+                             state_out, err, st, w_qdq != GDN_W_QDQ_NONE);
   if (dt == GDN_DTYPE_BF16)
     return launch_prefill_simt<__nv_bfloat16>(q, k, v, g, beta, state_in, cu_seqlens, n_seq, T,
                                               H, d_k, d_v, pk, kind, group, o, state_out, err,
@@ -581,6 +591,15 @@ gdn_status gdn_prefill(const void *q, const void *k, const void *v, const float 
                        void *cuda_stream) {
   return prefill_impl(q, k, v, g, beta, state_in, cu_seqlens, n_seq, T, H, d_k, d_v, dt, gk, qdq,
                       0, o, state_out, cuda_stream);
+}
+
+gdn_status gdn_prefill_w_qdq(const void *q, const void *k, const void *v, const float *g,
+                             const float *beta, const float *state_in, const int32_t *cu_seqlens,
+                             int n_seq, int T, int H, int d_k, int d_v, gdn_dtype dt,
+                             gdn_gate_kind gk, gdn_qdq_mode qdq, gdn_w_qdq_mode w_qdq, void *o,
+                             float *state_out, void *cuda_stream) {
+  return prefill_impl(q, k, v, g, beta, state_in, cu_seqlens, n_seq, T, H, d_k, d_v, dt, gk, qdq,
+                      0, o, state_out, cuda_stream, w_qdq);
 }
 
 gdn_status gdn_prefill_neumann(const void *q, const void *k, const void *v, const float *g,

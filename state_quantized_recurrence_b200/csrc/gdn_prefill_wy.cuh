@@ -63,6 +63,13 @@ constexpr uint32_t H_THI = 32768;   // (T diag(beta)) hi [t][t'] (B of U, K-majo
 constexpr uint32_t H_TLO = 40960;   // (T diag(beta)) lo
 constexpr uint32_t H_AQK = 49152;   // Aqk [t][t'] fp16 (B of O part 2, K-major)
 constexpr uint32_t kRxBytes = 57344;
+// With the FP8 QDQ of W: the W area holds the E4M3 codes of W, K-major
+// [t][k] (two 64-key halves 8 KB apart; B of X), and the 64 row scales at
+// H_WLO; 16,640 bytes of it are handed over.
+constexpr uint32_t H_WSC = H_WLO;
+constexpr uint32_t kWqBytes = 16384 + 256;
+constexpr uint32_t kRxBytesWq = kWqBytes + (kRxBytes - H_THI);
+constexpr int LDW = 129;  // row stride (floats) of W staged as fp32 [t][k] for the row amax
 
 // ---- chain CTA shared memory
 constexpr uint32_t C_KQ = 0;        // 2 x [K | gamma Q] fp16 (K h0 | Q h0 | K h1 | Q h1, 8 KB each)
@@ -259,6 +266,7 @@ __device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t (&v)[3
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+template <bool WQ>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 prefill_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ g,
@@ -345,7 +353,7 @@ prefill_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       for (int b = 0; b < 2; ++b) smc->qk_pend[b] = smc->v_pend[b] = smc->rx_pend[b] = 0;
       // chunks 0 and 1: both receive slots armed before the producer may copy
       for (int b = 0; b < 2 && b < n_chunks; ++b) {
-        sm100::mbar_arrive_expect_tx(&smc->rx_full[b], kRxBytes);
+        sm100::mbar_arrive_expect_tx(&smc->rx_full[b], WQ ? kRxBytesWq : kRxBytes);
         smc->rx_pend[b] = 1;
       }
     }
@@ -662,9 +670,9 @@ prefill_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       sm100::tc_fence_after();
       // K has been read: the buffer takes chunk j + 2
       if (tid == 0 && j + 2 < n_chunks && !sm->abort) issue_qk(j + 2);
-      // ---- W = sum of the two parts -> hi/lo [k][t] (B of the chain's X);
-      //      thread: key row `row`, tokens 32 wg .. + 31 ----
-      {
+      // ---- W = sum of the two parts; thread: key row `row`, tokens 32 wg .. + 31 ----
+      if (!WQ) {
+        // -> hi/lo [k][t] (B of the chain's X)
         float wa[32], wb[32];
         sm100::tmem_ld32(tmem + lane_off + TP_W + 32 * wg, wa);
         sm100::tmem_ld32(tmem + lane_off + TP_W + 64 + 32 * wg, wb);
@@ -672,13 +680,48 @@ prefill_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         for (int i = 0; i < 32; i += 2)
           f2_unpack(f2_add(f2_pack(wa[i], wa[i + 1]), f2_pack(wb[i], wb[i + 1])), wa[i], wa[i + 1]);
         store32_hl(stg + H_WHI, stg + H_WLO, row, 4 * wg, wa);
+      } else {
+        // FP8 QDQ of W, one scale per row (token) over the keys: W^T goes
+        // through the solve's scratch as fp32 [t][k] (stride LDW), each row
+        // is reduced by four threads (keys 32 q .. + 31), then coded
+        float *sW = reinterpret_cast<float *>(gbase + P_SA);
+        float *sRed = reinterpret_cast<float *>(gbase + P_SA) + 64 * LDW;
+        {
+          float wa[32], wb[32];
+          sm100::tmem_ld32(tmem + lane_off + TP_W + 32 * wg, wa);
+          sm100::tmem_ld32(tmem + lane_off + TP_W + 64 + 32 * wg, wb);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) sW[(32 * wg + i) * LDW + row] = wa[i] + wb[i];
+        }
+        __syncthreads();
+        const int t = tid & 63, qk = tid >> 6;  // row t, keys 32 qk .. + 31
+        float w[32];
+        float m = 0.f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          w[i] = sW[t * LDW + 32 * qk + i];
+          m = fmaxf(m, fabsf(w[i]));
+        }
+        sRed[qk * 64 + t] = m;
+        __syncthreads();
+        m = fmaxf(fmaxf(sRed[t], sRed[64 + t]), fmaxf(sRed[128 + t], sRed[192 + t]));
+        const ScaleRecip sr = make_scale(fp8_scale(m > 0.f ? m : 1.0f));
+        uint32_t c[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) c[i] = m > 0.f ? fp8_codes(w[2 * i], w[2 * i + 1], sr) : 0u;
+        const uint32_t half = stg + H_WHI + (uint32_t)(qk >> 1) * 8192u;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc)
+          st_shared_v4(sw128(half, t, 4 * (qk & 1) + cc), c[4 * cc], c[4 * cc + 1], c[4 * cc + 2],
+                       c[4 * cc + 3]);
+        if (qk == 0) reinterpret_cast<float *>(gbase + P_STG + b * kRxBytes + H_WSC)[t] = m > 0.f ? sr.s : 0.f;
       }
       sm100::fence_proxy_async();  // staging written by this CTA's threads -> bulk copy reads it
       sm100::tc_fence_before();
       __syncthreads();
       if (tid == 0 && !sm->abort)
-        sm100::bulk_copy_to_cluster(rx_buf_remote[b] + H_WHI, stg + H_WHI, H_THI - H_WHI,
-                                    rx_full_remote[b]);
+        sm100::bulk_copy_to_cluster(rx_buf_remote[b] + H_WHI, stg + H_WHI,
+                                    WQ ? kWqBytes : H_THI - H_WHI, rx_full_remote[b]);
     }
     // an aborted producer lets its TMA loads land before leaving
     if (tid == 0 && sm->abort) {
@@ -801,15 +844,31 @@ prefill_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         sm100::tc_fence_after();
         if (got && sm100::elect_one()) {
           if (!u_done) issue_u(it);
-#pragma unroll 1
-          for (int ks = 0; ks < 8; ++ks)
-            sm100::mma_f16_ts(tmem + TM_X, tmem + TM_S0C + 8u * ks,
-                              mndesc(rx + H_WHI + (uint32_t)ks * 2048u, 16384), ID_X, ks > 0);
-          if (!exact) {
+          if (!WQ) {
 #pragma unroll 1
             for (int ks = 0; ks < 8; ++ks)
-              sm100::mma_f16_ts(tmem + TM_X, tmem + TM_O2 + 8u * ks,
-                                mndesc(rx + H_WHI + (uint32_t)ks * 2048u, 16384), ID_X64, 1);
+              sm100::mma_f16_ts(tmem + TM_X, tmem + TM_S0C + 8u * ks,
+                                mndesc(rx + H_WHI + (uint32_t)ks * 2048u, 16384), ID_X, ks > 0);
+            if (!exact) {
+#pragma unroll 1
+              for (int ks = 0; ks < 8; ++ks)
+                sm100::mma_f16_ts(tmem + TM_X, tmem + TM_O2 + 8u * ks,
+                                  mndesc(rx + H_WHI + (uint32_t)ks * 2048u, 16384), ID_X64, 1);
+            }
+          } else {
+            // X = S0c Wc^T with the E4M3 codes of W (exact in fp16): one pass
+#pragma unroll 1
+            for (int ks = 0; ks < 8; ++ks)
+              sm100::mma_f16_ts(tmem + TM_X, tmem + TM_S0C + 8u * ks,
+                                kdesc(rx + H_WHI + (uint32_t)(ks >> 2) * 8192u + (uint32_t)(ks & 3) * 32u),
+                                ID_O, ks > 0);
+            if (!exact) {
+#pragma unroll 1
+              for (int ks = 0; ks < 8; ++ks)
+                sm100::mma_f16_ts(tmem + TM_X, tmem + TM_O2 + 8u * ks,
+                                  kdesc(rx + H_WHI + (uint32_t)(ks >> 2) * 8192u + (uint32_t)(ks & 3) * 32u),
+                                  ID_O, 1);
+            }
           }
           sm100::mma_commit(&sm->bar_x);
 #pragma unroll 1
@@ -857,7 +916,18 @@ prefill_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         sm100::tc_fence_after();
         float xa[32], xb[32], u[32];
         sm100::tmem_ld32(tmem + lane_off + TM_X + 32 * wg, xa);
-        sm100::tmem_ld32(tmem + lane_off + TM_X + 64 + 32 * wg, xb);
+        if (!WQ) {
+          sm100::tmem_ld32(tmem + lane_off + TM_X + 64 + 32 * wg, xb);
+        } else {
+          // the row scales of W: X a[t] * s_t, X b = 0
+          const float *wsc = reinterpret_cast<const float *>(gbase + C_RX + kb * kRxBytes + H_WSC) + 32 * wg;
+#pragma unroll
+          for (int t = 0; t < 32; t += 4) {
+            const float4 s4 = *reinterpret_cast<const float4 *>(wsc + t);
+            xa[t] *= s4.x; xa[t + 1] *= s4.y; xa[t + 2] *= s4.z; xa[t + 3] *= s4.w;
+            xb[t] = xb[t + 1] = xb[t + 2] = xb[t + 3] = 0.0f;
+          }
+        }
         sm100::tmem_ld32(tmem + lane_off + TM_U + 32 * wg, u);
         const uint64_t ms = f2_pack(-s0, -s0);
         uint32_t vh[16], dh[16], dl[16];
@@ -934,7 +1004,7 @@ prefill_wy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           // O part 2; this thread has seen those MMAs complete): arm it for
           // chunk it + 2, then hand it back to the producer
           if (it + 2 < n_chunks) {
-            sm100::mbar_arrive_expect_tx(&sm->rx_full[kb], kRxBytes);
+            sm100::mbar_arrive_expect_tx(&sm->rx_full[kb], WQ ? kRxBytesWq : kRxBytes);
             sm->rx_pend[kb] = 1 + (((it + 2) >> 1) & 1);
           }
           sm100::mbar_arrive_cluster_relaxed(rx_free_remote[kb]);

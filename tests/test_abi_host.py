@@ -38,6 +38,8 @@ def lib():
     L.gdn_prefill.restype = I
     L.gdn_prefill_neumann.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, P, P, P]
     L.gdn_prefill_neumann.restype = I
+    L.gdn_prefill_w_qdq.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, P, P, P]
+    L.gdn_prefill_w_qdq.restype = I
     L.gdn_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, P, P]
     L.gdn_decode.restype = I
     L.gdn_decode_packed.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, P]
@@ -99,6 +101,16 @@ def pn(lib, degree=3, **kw):
                                    a["stream"])
 
 
+def pw(lib, w_qdq=1, **kw):
+    a = dict(q=A, k=A, v=A, g=A, beta=A, state_in=None, cu=None, n_seq=2, T=64, H=4, d_k=128,
+             d_v=128, dt=BF16, gk=0, qdq=1, o=A, state_out=A, stream=None)
+    a.update(kw)
+    return lib.gdn_prefill_w_qdq(a["q"], a["k"], a["v"], a["g"], a["beta"], a["state_in"],
+                                 a["cu"], a["n_seq"], a["T"], a["H"], a["d_k"], a["d_v"],
+                                 a["dt"], a["gk"], a["qdq"], w_qdq, a["o"], a["state_out"],
+                                 a["stream"])
+
+
 def dc(lib, **kw):
     a = dict(q=A, k=A, v=A, g=A, beta=A, state=A, n_seq=2, H=4, d_k=128, d_v=128, dt=BF16, gk=0,
              qdq=2, o=A, stream=None)
@@ -127,7 +139,7 @@ def cv(lib, unpack=False, **kw):
                               a["d_v"], a["qdq"], a["stream"])
 
 
-@pytest.mark.parametrize("call", [pf, pn, dc, dp])
+@pytest.mark.parametrize("call", [pf, pn, pw, dc, dp])
 def test_validation_errors(lib, call):
     assert call(lib, n_seq=-1) == INVALID
     assert call(lib, H=0) == INVALID
@@ -151,6 +163,20 @@ def test_prefill_specific_errors(lib):
     assert pf(lib, state_out=A + 4) == INVALID
     assert pf(lib, state_in=A + 4) == INVALID
     assert pf(lib, cu=A + 2) == INVALID
+
+
+def test_w_qdq_unsupported_combinations(lib):
+    """The FP8 QDQ of W runs on the WY-form pair only: bf16, scalar gates,
+    d = 128, FP8 state tiles; anything else is refused before a launch (an
+    unknown W codec too)."""
+    assert pw(lib, w_qdq=2) == UNSUPPORTED
+    assert pw(lib, dt=F32) == UNSUPPORTED
+    assert pw(lib, gk=1) == UNSUPPORTED
+    assert pw(lib, d_k=64, d_v=64) == UNSUPPORTED
+    assert pw(lib, qdq=2) == UNSUPPORTED            # INT8 state
+    assert pw(lib, qdq=0) == UNSUPPORTED            # no state QDQ
+    assert pw(lib, n_seq=0) == OK
+    assert pw(lib, w_qdq=0, n_seq=0) == OK
 
 
 @pytest.mark.parametrize("degree", [-1, 0, 2, 4, 5, 30, 64, 127])
