@@ -129,13 +129,22 @@ __device__ __forceinline__ float qdq_int8(float x, const ScaleRecip &sr) {
   return __fmul_rn(c, sr.s);
 }
 
+// The two fp32 values of an fp16 pair (exact): mixed-precision adds of -0 on
+// the FMA pipe instead of two conversions.
+__device__ __forceinline__ void h2_to_f32(uint32_t h2, float &a, float &b) {
+  asm("{\n\t.reg .f16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "add.rn.f32.f16 %0, l, 0f80000000;\n\tadd.rn.f32.f16 %1, h, 0f80000000;\n\t}"
+      : "=f"(a), "=f"(b) : "r"(h2));
+}
+
 // E4M3 round trip of two values: RNE with saturation to +-448 (the
 // conversion's satfinite mode), then back to fp32 exactly.
 __device__ __forceinline__ float2 e4m3_round2(float a, float b) {
   __nv_fp8x2_storage_t p = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
   __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(p, __NV_E4M3);
-  __half2 hh = *reinterpret_cast<__half2 *>(&h);
-  return __half22float2(hh);
+  float2 r;
+  h2_to_f32(*reinterpret_cast<const uint32_t *>(&h), r.x, r.y);
+  return r;
 }
 
 // FP8 tile codec for two values sharing scale s > 0.
@@ -164,6 +173,29 @@ __device__ __forceinline__ float4 mul4(float4 c, float s) {
   return y;
 }
 
+// Integer-valued floats in [-2^22, 2^22] <-> their low byte / value through
+// the magic constant 1.5 * 2^23: adding it rounds to the nearest integer
+// (ties to even, the fp32 addition's own rounding) and leaves the integer in
+// the low mantissa bits, so neither direction needs a float <-> int
+// conversion instruction.
+constexpr float kMagicRound = 12582912.0f;  // 1.5 * 2^23
+// c = clamp(rint(q), -127, 127) as a float and as its two's-complement byte.
+__device__ __forceinline__ float int8_round_clamp(float q, uint32_t &byte) {
+  const float t = fminf(fmaxf(q, -127.0f), 127.0f) + kMagicRound;
+  byte = __float_as_uint(t) & 0xffu;
+  return t - kMagicRound;
+}
+// The signed value of byte `sel` (0..3) of w, as a float.
+template <int SEL>
+__device__ __forceinline__ float int8_byte_to_f32(uint32_t w) {
+  // prmt: result byte 0 is byte SEL of w, bytes 1-3 replicate its sign bit
+  // (selector nibbles with bit 3 set), i.e. the sign-extended integer
+  constexpr uint32_t kSel = SEL | ((8 | SEL) << 4) | ((8 | SEL) << 8) | ((8 | SEL) << 12);
+  int x;
+  asm("prmt.b32 %0, %1, 0, %2;" : "=r"(x) : "r"(w), "n"(kSel));
+  return __int_as_float(0x4B400000 + x) - kMagicRound;
+}
+
 __device__ __forceinline__ float int8_code(float x, const ScaleRecip &sr) {
   return fminf(fmaxf(rintf(div_by_scale(x, sr)), -127.0f), 127.0f);
 }
@@ -175,8 +207,9 @@ __device__ __forceinline__ unsigned short e4m3_code2(float x0, float x1, const S
 // Two E4M3 bytes (low byte first) -> their values, exactly.
 __device__ __forceinline__ float2 e4m3_pair_to_f2(unsigned short p) {
   __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)p, __NV_E4M3);
-  __half2 hh = *reinterpret_cast<__half2 *>(&h);
-  return __half22float2(hh);
+  float2 r;
+  h2_to_f32(*reinterpret_cast<const uint32_t *>(&h), r.x, r.y);
+  return r;
 }
 
 __device__ __forceinline__ float int8_scale(float amax) { return __fdiv_rn(amax, 127.0f); }

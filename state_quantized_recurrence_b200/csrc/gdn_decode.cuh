@@ -64,8 +64,8 @@ struct StateIO {
 #pragma unroll
         for (int j = 0; j < RPT; ++j) {
           const uint32_t w = cw[j];
-          h[j] = mul4(make_float4((float)(int8_t)(w & 0xffu), (float)(int8_t)((w >> 8) & 0xffu),
-                                  (float)(int8_t)((w >> 16) & 0xffu), (float)(int8_t)(w >> 24)),
+          h[j] = mul4(make_float4(int8_byte_to_f32<0>(w), int8_byte_to_f32<1>(w),
+                                  int8_byte_to_f32<2>(w), int8_byte_to_f32<3>(w)),
                       s[j]);
         }
       } else {
@@ -87,21 +87,53 @@ struct StateIO {
                                                    int warp, float *red, float4 (&h)[RPT]) {
     uint32_t cw[RPT];  // packed codes, 4 per row
     if (QK == kQdqInt8) {
+      // Row maxima over each group (GROUP / 4 consecutive lanes hold one
+      // group of a row); then each lane of a group computes the scale and
+      // reciprocal of the rows j = li, li + GL, ... (one IEEE division per
+      // lane instead of one per row) and the group's lanes exchange them.
+      constexpr int GL = GROUP / 4;
+      constexpr int SPL = (RPT + GL - 1) / GL;
+      const int li = lane % GL;
+      float m[RPT];
 #pragma unroll
       for (int j = 0; j < RPT; ++j) {
-        float m = fmaxf(fmaxf(fabsf(h[j].x), fabsf(h[j].y)), fmaxf(fabsf(h[j].z), fabsf(h[j].w)));
-        m = group_max<GROUP / 4>(m);  // a group spans GROUP / 4 consecutive lanes
+        float mj;
+        asm("max.f32 %0, %1, %2, %3;" : "=f"(mj) : "f"(fabsf(h[j].x)), "f"(fabsf(h[j].y)),
+            "f"(fmaxf(fabsf(h[j].z), fabsf(h[j].w))));
+        m[j] = group_max<GL>(mj);
+      }
+      float s_own[SPL], r_own[SPL];
+#pragma unroll
+      for (int i = 0; i < SPL; ++i) {
+        float ms = 0.0f;
+#pragma unroll
+        for (int j = i * GL; j < RPT && j < (i + 1) * GL; ++j) ms = (li == j - i * GL) ? m[j] : ms;
+        const ScaleRecip so = make_scale(int8_scale(ms > 0.0f ? ms : 1.0f));
+        s_own[i] = so.s;
+        r_own[i] = so.r;
+      }
+#pragma unroll
+      for (int j = 0; j < RPT; ++j) {
+        const int src = (lane & ~(GL - 1)) | (j % GL);
+        ScaleRecip s;
+        s.s = __shfl_sync(0xffffffffu, s_own[j / GL], src);
+        s.r = __shfl_sync(0xffffffffu, r_own[j / GL], src);
+        s.pre = s.s < 0x1p-100f ? 0x1p64f : 1.0f;
+        s.s2 = __fmul_rn(s.s, s.pre);
         float sc = 0.0f;
-        if (m == 0.0f) {
+        if (m[j] == 0.0f) {
           h[j] = make_float4(0.f, 0.f, 0.f, 0.f);
           cw[j] = 0u;
         } else {
-          const ScaleRecip s = make_scale(int8_scale(m));
           sc = s.s;
-          const float4 c = int8_code4(h[j], s);
+          float q0, q1, q2, q3;
+          div_by_scale2(h[j].x, h[j].y, s, q0, q1);
+          div_by_scale2(h[j].z, h[j].w, s, q2, q3);
+          uint32_t b0, b1, b2, b3;
+          const float4 c = make_float4(int8_round_clamp(q0, b0), int8_round_clamp(q1, b1),
+                                       int8_round_clamp(q2, b2), int8_round_clamp(q3, b3));
           if (PACKED) {
-            cw[j] = ((uint32_t)(uint8_t)(int8_t)c.x) | ((uint32_t)(uint8_t)(int8_t)c.y << 8) |
-                    ((uint32_t)(uint8_t)(int8_t)c.z << 16) | ((uint32_t)(uint8_t)(int8_t)c.w << 24);
+            cw[j] = __byte_perm(b0 | (b1 << 8), b2 | (b3 << 8), 0x5410);
           } else {
             h[j] = mul4(c, s.s);
           }

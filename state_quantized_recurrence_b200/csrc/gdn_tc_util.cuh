@@ -41,13 +41,6 @@ __device__ __forceinline__ float sub_h_hi(float x, uint32_t h2) {
       "fma.rn.f32.f16 %0, h, m, %2;\n\t}" : "=f"(d) : "r"(h2), "f"(x));
   return d;
 }
-// The two fp32 values of an fp16 pair (exact): mixed-precision adds of -0.
-__device__ __forceinline__ void h2_to_f32(uint32_t h2, float &a, float &b) {
-  asm("{\n\t.reg .f16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
-      "add.rn.f32.f16 %0, l, 0f80000000;\n\tadd.rn.f32.f16 %1, h, 0f80000000;\n\t}"
-      : "=f"(a), "=f"(b) : "r"(h2));
-}
-
 // hi = fp16(x), lo = fp16(x - hi), packed in pairs (x - hi is exact in fp32).
 __device__ __forceinline__ void split_h2(float a, float b, uint32_t &hi, uint32_t &lo) {
   hi = pack_h2(a, b);
