@@ -185,15 +185,45 @@ __device__ __forceinline__ float int8_round_clamp(float q, uint32_t &byte) {
   byte = __float_as_uint(t) & 0xffu;
   return t - kMagicRound;
 }
-// The signed value of byte `sel` (0..3) of w, as a float.
-template <int SEL>
-__device__ __forceinline__ float int8_byte_to_f32(uint32_t w) {
-  // prmt: result byte 0 is byte SEL of w, bytes 1-3 replicate its sign bit
-  // (selector nibbles with bit 3 set), i.e. the sign-extended integer
-  constexpr uint32_t kSel = SEL | ((8 | SEL) << 4) | ((8 | SEL) << 8) | ((8 | SEL) << 12);
-  int x;
-  asm("prmt.b32 %0, %1, 0, %2;" : "=r"(x) : "r"(w), "n"(kSel));
-  return __int_as_float(0x4B400000 + x) - kMagicRound;
+
+// The four INT8 codes in the bytes of w (two's complement), exactly, as
+// floats: flipping each byte's sign bit gives u = c + 128 in 0 .. 255, prmt
+// puts u under the upper bytes of 1.5 * 2^23 (the float 1.5 * 2^23 + u, an
+// integer where the fp32 ulp is 1), and one packed subtraction of
+// 1.5 * 2^23 + 128 leaves c.
+__device__ __forceinline__ float4 int8x4_to_f32(uint32_t w) {
+  const uint32_t u = w ^ 0x80808080u;
+  uint32_t b0, b1, b2, b3;
+  asm("prmt.b32 %0, %1, 0x4B400000, 0x7650;" : "=r"(b0) : "r"(u));
+  asm("prmt.b32 %0, %1, 0x4B400000, 0x7651;" : "=r"(b1) : "r"(u));
+  asm("prmt.b32 %0, %1, 0x4B400000, 0x7652;" : "=r"(b2) : "r"(u));
+  asm("prmt.b32 %0, %1, 0x4B400000, 0x7653;" : "=r"(b3) : "r"(u));
+  const uint64_t off = f2_pack(-(kMagicRound + 128.0f), -(kMagicRound + 128.0f));
+  float4 c;
+  f2_unpack(f2_add(f2_pack(__uint_as_float(b0), __uint_as_float(b1)), off), c.x, c.y);
+  f2_unpack(f2_add(f2_pack(__uint_as_float(b2), __uint_as_float(b3)), off), c.z, c.w);
+  return c;
+}
+
+// INT8 codes of four quotients q = x / s already correctly rounded, with
+// s = RN(amax / 127) of a group whose |x| <= amax: then |x| / s <=
+// 127 / (1 - 2^-24) < 127 + 2^-16, so RN(q) stays below 127.5 and rounding to
+// the nearest integer lands in [-127, 127] by itself; the codec's clamp is
+// the identity there and is left out.  Returns the codes' two's-complement
+// bytes packed low byte first; c receives the codes as floats.
+__device__ __forceinline__ uint32_t int8_round4(uint64_t q01, uint64_t q23, float4 &c) {
+  const uint64_t m2 = f2_pack(kMagicRound, kMagicRound);
+  float t0, t1, t2, t3;
+  f2_unpack(f2_add(q01, m2), t0, t1);
+  f2_unpack(f2_add(q23, m2), t2, t3);
+  uint32_t lo, hi, w;
+  asm("prmt.b32 %0, %1, %2, 0x3340;" : "=r"(lo) : "r"(__float_as_uint(t0)), "r"(__float_as_uint(t1)));
+  asm("prmt.b32 %0, %1, %2, 0x4033;" : "=r"(hi) : "r"(__float_as_uint(t2)), "r"(__float_as_uint(t3)));
+  asm("prmt.b32 %0, %1, %2, 0x7610;" : "=r"(w) : "r"(lo), "r"(hi));
+  const uint64_t nm2 = f2_pack(-kMagicRound, -kMagicRound);
+  f2_unpack(f2_add(f2_pack(t0, t1), nm2), c.x, c.y);
+  f2_unpack(f2_add(f2_pack(t2, t3), nm2), c.z, c.w);
+  return w;
 }
 
 __device__ __forceinline__ float int8_code(float x, const ScaleRecip &sr) {

@@ -42,9 +42,67 @@ struct StateRef {
   float *scales;   // packed storage: INT8 [d_k, d_v / GROUP], FP8 [d_v / 64]
 };
 
+// Reduce-scatter of row maxima over the 2 D lanes of a group: on entry w
+// holds this lane's maxima of K rows; each exchange at lane distance d
+// halves the rows a lane keeps (the upper half where bit d of its lane index
+// is set) and merges in its partner's maxima of them, until SPL rows are
+// left; further exchanges only merge.  On exit w[0 .. SPL) are the group
+// maxima of the rows scatter_owner names.
+template <int D, int K, int SPL, int N>
+__device__ __forceinline__ void scatter_max(float (&w)[N], int li) {
+  if constexpr (D >= 1) {
+    if constexpr (K > SPL) {
+      const bool up = (li & D) != 0;
+#pragma unroll
+      for (int i = 0; i < K / 2; ++i) {
+        const float send = up ? w[i] : w[i + K / 2];
+        const float keep = up ? w[i + K / 2] : w[i];
+        w[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, D));
+      }
+      scatter_max<D / 2, K / 2, SPL, N>(w, li);
+    } else {
+#pragma unroll
+      for (int i = 0; i < SPL; ++i) w[i] = fmaxf(w[i], __shfl_xor_sync(0xffffffffu, w[i], D));
+      scatter_max<D / 2, K, SPL, N>(w, li);
+    }
+  }
+}
+// The lane (within its group) that holds row j's group maximum after
+// scatter_max<D, K, SPL>, in slot j % SPL: the halving exchanges map row bit
+// K / 2 to lane bit D, row bit K / 4 to lane bit D / 2, and so on.
+template <int D, int K, int SPL>
+__host__ __device__ constexpr int scatter_owner(int j) {
+  if constexpr (D >= 1 && K > SPL)
+    return ((j & (K / 2)) ? D : 0) + scatter_owner<D / 2, K / 2, SPL>(j);
+  else
+    return 0;
+}
+
 template <int DK, int DV, int QK, int GROUP, bool PACKED>
 struct StateIO {
   static constexpr int RPT = DK / 16;  // state rows per thread
+
+  // The fp32 values code * scale of a thread's packed codes: cw[j] holds
+  // the four codes of row rg + 16 j, sc[j] its INT8 group scale (FP8: sc[0]
+  // is the tile scale).
+  __device__ __forceinline__ static void dequant(const uint32_t (&cw)[RPT], const float (&sc)[RPT],
+                                                 float4 (&h)[RPT]) {
+    if (QK == kQdqInt8) {
+#pragma unroll
+      for (int j = 0; j < RPT; ++j) {
+        const uint32_t w = cw[j];
+        h[j] = mul4(int8x4_to_f32(w), sc[j]);
+      }
+    } else {
+      const float st = sc[0];
+#pragma unroll
+      for (int j = 0; j < RPT; ++j) {
+        const float2 lo = e4m3_pair_to_f2((unsigned short)(cw[j] & 0xffffu));
+        const float2 hi = e4m3_pair_to_f2((unsigned short)(cw[j] >> 16));
+        h[j] = mul4(make_float4(lo.x, lo.y, hi.x, hi.y), st);
+      }
+    }
+  }
 
   // Row `r`, columns col .. col+3 of the state, as fp32 values.
   __device__ __forceinline__ static void load(const StateRef &sr, int rg, int col, float4 (&h)[RPT]) {
@@ -58,26 +116,11 @@ struct StateIO {
 #pragma unroll
       for (int j = 0; j < RPT; ++j)
         cw[j] = __ldcs(reinterpret_cast<const unsigned int *>(sr.codes + (rg + 16 * j) * DV + col));
-      if (QK == kQdqInt8) {
 #pragma unroll
-        for (int j = 0; j < RPT; ++j) s[j] = __ldg(sr.scales + (rg + 16 * j) * (DV / GROUP) + col / GROUP);
-#pragma unroll
-        for (int j = 0; j < RPT; ++j) {
-          const uint32_t w = cw[j];
-          h[j] = mul4(make_float4(int8_byte_to_f32<0>(w), int8_byte_to_f32<1>(w),
-                                  int8_byte_to_f32<2>(w), int8_byte_to_f32<3>(w)),
-                      s[j]);
-        }
-      } else {
-        const float st = __ldg(sr.scales + col / 64);
-#pragma unroll
-        for (int j = 0; j < RPT; ++j) {
-          const float2 lo = e4m3_pair_to_f2((unsigned short)(cw[j] & 0xffffu));
-          const float2 hi = e4m3_pair_to_f2((unsigned short)(cw[j] >> 16));
-          h[j] = make_float4(__fmul_rn(lo.x, st), __fmul_rn(lo.y, st), __fmul_rn(hi.x, st),
-                             __fmul_rn(hi.y, st));
-        }
-      }
+      for (int j = 0; j < RPT; ++j)
+        s[j] = QK == kQdqInt8 ? __ldg(sr.scales + (rg + 16 * j) * (DV / GROUP) + col / GROUP)
+                              : (j == 0 ? __ldg(sr.scales + col / 64) : 0.0f);
+      dequant(cw, s, h);
     }
   }
 
@@ -88,58 +131,69 @@ struct StateIO {
     uint32_t cw[RPT];  // packed codes, 4 per row
     if (QK == kQdqInt8) {
       // Row maxima over each group (GROUP / 4 consecutive lanes hold one
-      // group of a row); then each lane of a group computes the scale and
-      // reciprocal of the rows j = li, li + GL, ... (one IEEE division per
-      // lane instead of one per row) and the group's lanes exchange them.
+      // group of a row), reduced and scattered at once: after the exchange
+      // each lane holds the group maxima of SPL rows (scatter_max), computes
+      // their scales and reciprocals (one IEEE division per lane, not per
+      // row), and the group's lanes fetch them back row by row.
       constexpr int GL = GROUP / 4;
-      constexpr int SPL = (RPT + GL - 1) / GL;
+      constexpr int SPL = RPT / GL > 0 ? RPT / GL : 1;
       const int li = lane % GL;
       float m[RPT];
 #pragma unroll
-      for (int j = 0; j < RPT; ++j) {
-        float mj;
-        asm("max.f32 %0, %1, %2, %3;" : "=f"(mj) : "f"(fabsf(h[j].x)), "f"(fabsf(h[j].y)),
+      for (int j = 0; j < RPT; ++j)
+        asm("max.f32 %0, %1, %2, %3;" : "=f"(m[j]) : "f"(fabsf(h[j].x)), "f"(fabsf(h[j].y)),
             "f"(fmaxf(fabsf(h[j].z), fabsf(h[j].w))));
-        m[j] = group_max<GL>(mj);
-      }
+      scatter_max<GL / 2, RPT, SPL>(m, li);
+      // s = amax / 127 (0 for an all-zero group, whose values are all +-0 and
+      // give code 0 with any finite reciprocal); r = RN(1 / s), 1 for an
+      // all-zero group and +inf where amax / 127 underflows to 0
       float s_own[SPL], r_own[SPL];
+      bool tiny = false;
 #pragma unroll
       for (int i = 0; i < SPL; ++i) {
-        float ms = 0.0f;
-#pragma unroll
-        for (int j = i * GL; j < RPT && j < (i + 1) * GL; ++j) ms = (li == j - i * GL) ? m[j] : ms;
-        const ScaleRecip so = make_scale(int8_scale(ms > 0.0f ? ms : 1.0f));
-        s_own[i] = so.s;
-        r_own[i] = so.r;
+        s_own[i] = int8_scale(m[i]);
+        r_own[i] = s_own[i] > 0.0f ? __frcp_rn(s_own[i]) : (m[i] > 0.0f ? __int_as_float(0x7f800000) : 1.0f);
+        tiny |= m[i] > 0.0f && s_own[i] < 0x1p-100f;
       }
+      // A scale below 2^-100 (or one that underflowed) takes the scalar
+      // codec's steps: the pre-scaled quotient and the clamp, which such a
+      // scale needs since its relative rounding error is not bounded by
+      // 2^-24.  Every other row divides directly, and |x| / s < 127 + 2^-16
+      // makes its clamp the identity (int8_round4).
+      const bool any_tiny = __any_sync(0xffffffffu, tiny);
 #pragma unroll
       for (int j = 0; j < RPT; ++j) {
-        const int src = (lane & ~(GL - 1)) | (j % GL);
-        ScaleRecip s;
-        s.s = __shfl_sync(0xffffffffu, s_own[j / GL], src);
-        s.r = __shfl_sync(0xffffffffu, r_own[j / GL], src);
-        s.pre = s.s < 0x1p-100f ? 0x1p64f : 1.0f;
-        s.s2 = __fmul_rn(s.s, s.pre);
-        float sc = 0.0f;
-        if (m[j] == 0.0f) {
-          h[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-          cw[j] = 0u;
+        const int src = (lane & ~(GL - 1)) | scatter_owner<GL / 2, RPT, SPL>(j);
+        const float sj = __shfl_sync(0xffffffffu, s_own[j % SPL], src);
+        const float rj = __shfl_sync(0xffffffffu, r_own[j % SPL], src);
+        uint64_t q01, q23;
+        if (!any_tiny) {
+          const uint64_t rr = f2_pack(rj, rj), ns = f2_pack(-sj, -sj);
+          const uint64_t x01 = f2_pack(h[j].x, h[j].y), x23 = f2_pack(h[j].z, h[j].w);
+          q01 = f2_mul(x01, rr);
+          q23 = f2_mul(x23, rr);
+          q01 = f2_fma(f2_fma(q01, ns, x01), rr, q01);
+          q23 = f2_fma(f2_fma(q23, ns, x23), rr, q23);
         } else {
-          sc = s.s;
-          float q0, q1, q2, q3;
-          div_by_scale2(h[j].x, h[j].y, s, q0, q1);
-          div_by_scale2(h[j].z, h[j].w, s, q2, q3);
-          uint32_t b0, b1, b2, b3;
-          const float4 c = make_float4(int8_round_clamp(q0, b0), int8_round_clamp(q1, b1),
-                                       int8_round_clamp(q2, b2), int8_round_clamp(q3, b3));
-          if (PACKED) {
-            cw[j] = __byte_perm(b0 | (b1 << 8), b2 | (b3 << 8), 0x5410);
-          } else {
-            h[j] = mul4(c, s.s);
-          }
+          ScaleRecip sr;
+          sr.s = sj;
+          sr.pre = sj < 0x1p-100f ? 0x1p64f : 1.0f;
+          sr.s2 = __fmul_rn(sj, sr.pre);
+          sr.r = sr.pre == 1.0f ? rj : __frcp_rn(sr.s2);
+          float q[4];
+          div_by_scale2(h[j].x, h[j].y, sr, q[0], q[1]);
+          div_by_scale2(h[j].z, h[j].w, sr, q[2], q[3]);
+          const bool zero_row = sj == 0.0f && rj == 1.0f;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) q[e] = zero_row ? 0.0f : fminf(fmaxf(q[e], -127.0f), 127.0f);
+          q01 = f2_pack(q[0], q[1]);
+          q23 = f2_pack(q[2], q[3]);
         }
+        float4 c;
+        cw[j] = int8_round4(q01, q23, c);
+        if (!PACKED) h[j] = mul4(c, sj);
         if (PACKED && (col % GROUP) == 0)
-          sr.scales[(rg + 16 * j) * (DV / GROUP) + col / GROUP] = sc;
+          sr.scales[(rg + 16 * j) * (DV / GROUP) + col / GROUP] = sj;
       }
     } else if (QK == kQdqFp8Tile) {
       float m = 0.0f;
@@ -162,12 +216,19 @@ struct StateIO {
         const ScaleRecip s = make_scale(fp8_scale(m));
 #pragma unroll
         for (int j = 0; j < RPT; ++j) {
+          // the quotients in packed pairs (the scalar codec's roundings)
+          float q0, q1, q2, q3;
+          div_by_scale2(h[j].x, h[j].y, s, q0, q1);
+          div_by_scale2(h[j].z, h[j].w, s, q2, q3);
+          const unsigned short lo = (unsigned short)__nv_cvt_float2_to_fp8x2(
+              make_float2(q0, q1), __NV_SATFINITE, __NV_E4M3);
+          const unsigned short hi = (unsigned short)__nv_cvt_float2_to_fp8x2(
+              make_float2(q2, q3), __NV_SATFINITE, __NV_E4M3);
           if (PACKED) {
-            cw[j] = (uint32_t)e4m3_code2(h[j].x, h[j].y, s) | ((uint32_t)e4m3_code2(h[j].z, h[j].w, s) << 16);
+            cw[j] = (uint32_t)lo | ((uint32_t)hi << 16);
           } else {
-            const float2 lo = qdq_fp8_2(h[j].x, h[j].y, s);
-            const float2 hi = qdq_fp8_2(h[j].z, h[j].w, s);
-            h[j] = make_float4(lo.x, lo.y, hi.x, hi.y);
+            const float2 a = e4m3_pair_to_f2(lo), b = e4m3_pair_to_f2(hi);
+            h[j] = mul4(make_float4(a.x, a.y, b.x, b.y), s.s);
           }
         }
       }

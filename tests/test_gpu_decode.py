@@ -221,15 +221,18 @@ def test_decode_single_head_edge(cuda_lib):
                                rtol=1e-5, atol=1e-7)
 
 
-@pytest.mark.parametrize("mode", ["int8_g32", "fp8_tile64"])
-def test_decode_codec_bit_exact_wide_range(cuda_lib, mode):
-    """4 M state values whose groups span 2^-140 .. 2^60 in magnitude: the
+@pytest.mark.parametrize("mode", ["int8_g32", "int8_g16", "fp8_tile64"])
+@pytest.mark.parametrize("lo_exp", [-140, -90])
+def test_decode_codec_bit_exact_wide_range(cuda_lib, mode, lo_exp):
+    """4 M state values whose groups span 2^lo_exp .. 2^60 in magnitude: the
     codec (scale, quotient, rounding, dequantization) is bit-exact against
-    the oracle's IEEE fp32 codec everywhere, tiny scales included."""
+    the oracle's IEEE fp32 codec everywhere.  From 2^-140 most warps hold a
+    scale below 2^-100 and take the pre-scaled quotient; from 2^-90 none
+    does and every warp divides directly."""
     gen = torch.Generator().manual_seed(123)
     N, H, dk, dv = 16, 16, 128, 128
     st = torch.randn((N, H, dk, dv), generator=gen)
-    expo = torch.randint(-140, 60, (N, H, dk, dv // 32), generator=gen).float()
+    expo = torch.randint(lo_exp, 60, (N, H, dk, dv // 32), generator=gen).float()
     st = (st * torch.exp2(expo).repeat_interleave(32, dim=-1)).float()
     q = torch.randn((N, H, dk), generator=gen).to(torch.bfloat16)
     v = torch.randn((N, H, dv), generator=gen).to(torch.bfloat16)

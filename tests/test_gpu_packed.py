@@ -127,3 +127,31 @@ def test_packed_empty_batch(cuda_lib):
     o = sqr.gdn_decode_packed(e, e, e, torch.empty((0, 2), device="cuda"),
                               torch.empty((0, 2), device="cuda"), ps)
     assert o.shape == (0, 2, 128)
+
+
+@pytest.mark.parametrize("mode", ["fp8_tile64", "int8_g32"])
+def test_decode_packed_unaligned_storage(cuda_lib, mode):
+    """Codes and scales at 4-byte (not 16-byte) offsets, the alignment the
+    C ABI accepts: results stay bit-identical to the fp32 storage and no byte
+    outside the codes is written."""
+    sqr = cuda_lib
+    N, H, d_k, d_v = 7, 5, 128, 128
+    x = make_states(N, H, d_k, d_v, seed=31).cuda()
+    ps = sqr.gdn_state_pack(x, mode)
+    state = sqr.gdn_state_unpack(ps)
+    cbuf = torch.zeros(ps.codes.numel() + 16, dtype=torch.uint8, device="cuda")
+    sbuf = torch.zeros(ps.scales.numel() + 4, dtype=torch.float32, device="cuda")
+    codes = cbuf[4:4 + ps.codes.numel()].view(ps.codes.shape)
+    scales = sbuf[1:1 + ps.scales.numel()].view(ps.scales.shape)
+    assert codes.data_ptr() % 16 == 4 and scales.data_ptr() % 16 == 4
+    codes.copy_(ps.codes)
+    scales.copy_(ps.scales)
+    pu = sqr.PackedState(codes, scales, mode)
+    for q, k, v, g, beta in decode_inputs(N, H, d_k, d_v, "bf16", "scalar", 3, seed=32):
+        o32 = sqr.gdn_decode(q, k, v, g, beta, state, qdq=mode)
+        opk = sqr.gdn_decode_packed(q, k, v, g, beta, pu)
+        assert torch.equal(o32, opk)
+    torch.cuda.synchronize()
+    assert torch.equal(sqr.gdn_state_unpack(pu), state)
+    assert torch.equal(cbuf[:4], torch.zeros(4, dtype=torch.uint8, device="cuda"))
+    assert torch.equal(cbuf[4 + ps.codes.numel():], torch.zeros(12, dtype=torch.uint8, device="cuda"))
