@@ -780,12 +780,17 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       sm100::tc_fence_after();
       if (tid == 0 && !sm->abort) {
         // MMAs 3 and 4 have read the received tiles: arm the next chunk's
-        // transfer, then release the buffer to the producer
+        // transfer, then release the buffer to the producer.  A relaxed
+        // arrive: what the producer must not overtake are the tensor-core
+        // reads of the buffer, which the commit barrier this thread has
+        // waited for already orders; no thread of this CTA writes the buffer
+        // (a release arrive would also wait for this thread's outstanding
+        // stores of the previous chunk's outputs).
         if (!last) {
           sm100::mbar_arrive_expect_tx(&sm->rx_full, kRxBytes);
           sm->rx_pend = 1 + ((it + 1) & 1);
         }
-        sm100::mbar_arrive_cluster(rx_free_remote);
+        sm100::mbar_arrive_cluster_relaxed(rx_free_remote);
       }
       // the buffer MMA 5 just released takes the chunk after next
       if (tid == 128 && !last && it + 2 < n_chunks && !sm->abort) issue_qk(tb + 2 * kC, it + 2);
@@ -798,7 +803,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             float y[32];
             sm100::tmem_ld32(tmem + lane_off + TM_D4 + 64 * wg + 32 * p, y);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) mh = fmaxf(mh, fabsf(y[i]));
+            for (int i = 0; i < 32; i += 2) mh = max_abs2(mh, y[i], y[i + 1]);
           }
         }
         if (QK == kQdqFp8Tile) {
@@ -809,6 +814,9 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
         const float gn_next = last ? 1.0f : gt_next->gn_exp;
         const ScaleRecip sr_tile = make_scale(fp8_scale(QK == kQdqFp8Tile && mh > 0.f ? mh : 1.0f));
+        // FP8: the dequantized codes go straight into the next carry's accumulator
+        // (code x (s gamma_n), one rounding); the last chunk's are the state itself
+        const float sdq = last ? sr_tile.s : sr_tile.s * gn_next;
 #pragma unroll
         for (int p = 0; p < 2; ++p) {
           const int c0v = 64 * wg + 32 * p;
@@ -824,12 +832,12 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             } else if (sr_tile.pre == 1.0f) {
 #pragma unroll
               for (int i = 0; i < 32; i += 2)
-                code[i >> 1] = fp8_code_pair(y[i], y[i + 1], sr_tile.s, sr_tile.r, y[i], y[i + 1]);
+                code[i >> 1] = fp8_code_pair(y[i], y[i + 1], sr_tile.s, sr_tile.r, y[i], y[i + 1], sdq);
             } else {
 #pragma unroll
               for (int i = 0; i < 32; i += 2)
                 code[i >> 1] = fp8_code_pair(y[i] * sr_tile.pre, y[i + 1] * sr_tile.pre, sr_tile.s2,
-                                             sr_tile.r, y[i], y[i + 1], sr_tile.s);
+                                             sr_tile.r, y[i], y[i + 1], sdq);
             }
 #pragma unroll
             for (int c = 0; c < 4; ++c)
@@ -865,7 +873,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             for (int i = 0; i < 32; i += 4)
               *reinterpret_cast<float4 *>(dst + i) = make_float4(y[i], y[i + 1], y[i + 2], y[i + 3]);
           } else {
-            scale32(y, gn_next);
+            if (QK != kQdqFp8Tile) scale32(y, gn_next);
             sm100::tmem_st32(tmem + lane_off + TM_D4 + c0v, y);
           }
         }

@@ -705,7 +705,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           float y[32];
           sm100::tmem_ld32(tmem + lane_off + TM_D4 + 64 * wg + 32 * p, y);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) mh = fmaxf(mh, fabsf(y[i]));
+          for (int i = 0; i < 32; i += 2) mh = max_abs2(mh, y[i], y[i + 1]);
         }
       }
       if (QK == kQdqFp8Tile) {
@@ -716,6 +716,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       }
       const float gn_next = last ? 1.0f : sm->gt[(it + 1) & 1].gn_exp;
       const ScaleRecip sr_tile = make_scale(fp8_scale(QK == kQdqFp8Tile && mh > 0.f ? mh : 1.0f));
+      // FP8: the dequantized codes go straight into the next carry's accumulator
+      // (code x (s gamma_n), one rounding); the last chunk's are the state itself
+      const float sdq = last ? sr_tile.s : sr_tile.s * gn_next;
       // Pass 2: quantize; H0 operand tiles (exact codes for FP8, hi/lo
       // otherwise); gamma_n(next) * H into TMEM as the next carry's
       // accumulator; state_out after the last chunk.
@@ -734,12 +737,12 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           } else if (sr_tile.pre == 1.0f) {
 #pragma unroll
             for (int i = 0; i < 32; i += 2)
-              code[i >> 1] = fp8_code_pair(y[i], y[i + 1], sr_tile.s, sr_tile.r, y[i], y[i + 1]);
+              code[i >> 1] = fp8_code_pair(y[i], y[i + 1], sr_tile.s, sr_tile.r, y[i], y[i + 1], sdq);
           } else {
 #pragma unroll
             for (int i = 0; i < 32; i += 2)
               code[i >> 1] = fp8_code_pair(y[i] * sr_tile.pre, y[i + 1] * sr_tile.pre, sr_tile.s2,
-                                           sr_tile.r, y[i], y[i + 1], sr_tile.s);
+                                           sr_tile.r, y[i], y[i + 1], sdq);
           }
 #pragma unroll
           for (int c = 0; c < 4; ++c)
@@ -776,7 +779,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           for (int i = 0; i < 32; i += 4)
             *reinterpret_cast<float4 *>(dst + i) = make_float4(y[i], y[i + 1], y[i + 2], y[i + 3]);
         } else {
-          scale32(y, gn_next);
+          if (QK != kQdqFp8Tile) scale32(y, gn_next);
           sm100::tmem_st32(tmem + lane_off + TM_D4 + c0v, y);
         }
       }

@@ -85,10 +85,10 @@ __device__ __forceinline__ void scale32(float *y, float s) {
 
 // E4M3 codes of x0/s2 and x1/s2 (correctly rounded quotients from r = RN(1/s2),
 // Markstein's correction), returned as an fp16 pair (exact); y0, y1 receive
-// the dequantized values code * s (s = s2 unless the operands were
-// pre-scaled by a power of two).
+// code * sd (the dequantized values for sd = the scale, possibly times a
+// decay).  The fp16 -> fp32 widening runs on the FMA pipe (h2_to_f32).
 __device__ __forceinline__ uint32_t fp8_code_pair(float x0, float x1, float s2, float r, float &y0,
-                                                  float &y1, float s = 0.0f) {
+                                                  float &y1, float sd) {
   const uint64_t x = f2_pack(x0, x1), rr = f2_pack(r, r);
   const uint64_t q = f2_mul(x, rr);
   const uint64_t t = f2_fma(f2_fma(q, f2_pack(-s2, -s2), x), rr, q);
@@ -97,11 +97,18 @@ __device__ __forceinline__ uint32_t fp8_code_pair(float x0, float x1, float s2, 
   const __nv_fp8x2_storage_t f8 =
       __nv_cvt_float2_to_fp8x2(make_float2(t0, t1), __NV_SATFINITE, __NV_E4M3);
   const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(f8, __NV_E4M3);
-  const __half2 hh = *reinterpret_cast<const __half2 *>(&hr);
-  const float2 cf = __half22float2(hh);
-  const float sd = s == 0.0f ? s2 : s;
-  f2_unpack(f2_mul(f2_pack(cf.x, cf.y), f2_pack(sd, sd)), y0, y1);
-  return *reinterpret_cast<const uint32_t *>(&hh);
+  const uint32_t h2 = *reinterpret_cast<const uint32_t *>(&hr);
+  float c0, c1;
+  h2_to_f32(h2, c0, c1);
+  f2_unpack(f2_mul(f2_pack(c0, c1), f2_pack(sd, sd)), y0, y1);
+  return h2;
+}
+
+// max(m, |a|, |b|) in one three-input max.
+__device__ __forceinline__ float max_abs2(float m, float a, float b) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(m), "f"(fabsf(a)), "f"(fabsf(b)));
+  return d;
 }
 
 // In-place bf16 -> fp16 conversion of half `part` (the key columns
