@@ -296,16 +296,36 @@ __device__ __forceinline__ void decode_slab(float4 (&h)[DK / 16], const float *s
     red_b[warp][cq] = make_float4(pb[0], pb[1], pb[2], pb[3]);
   }
   __syncthreads();
-  float a[4] = {0.f, 0.f, 0.f, 0.f}, b[4] = {0.f, 0.f, 0.f, 0.f};
+  // the 8 warps' partial sums, in warp order (packed pairs, the scalar
+  // additions' roundings), formed once per column by warp 0 (lanes 0-15: a,
+  // 16-31: b) into row 0 and read back by every thread
+  if (warp == 0) {
+    float4(*red)[16] = lane < 16 ? red_a : red_b;
+    const int c = lane & 15;
+    uint64_t s01 = 0, s23 = 0;
 #pragma unroll
-  for (int w = 0; w < 8; ++w) {
-    const float4 x = red_a[w][cq], y = red_b[w][cq];
-    a[0] += x.x; a[1] += x.y; a[2] += x.z; a[3] += x.w;
-    b[0] += y.x; b[1] += y.y; b[2] += y.z; b[3] += y.w;
+    for (int w = 0; w < 8; ++w) {
+      const float4 x = red[w][c];
+      s01 = f2_add(s01, f2_pack(x.x, x.y));
+      s23 = f2_add(s23, f2_pack(x.z, x.w));
+    }
+    float4 r;
+    f2_unpack(s01, r.x, r.y);
+    f2_unpack(s23, r.z, r.w);
+    red[0][c] = r;
   }
-  float u[4];
-  u[0] = bt * (v4.x - a[0]); u[1] = bt * (v4.y - a[1]);
-  u[2] = bt * (v4.z - a[2]); u[3] = bt * (v4.w - a[3]);
+  __syncthreads();
+  const float4 sa = red_a[0][cq], sb = red_b[0][cq];
+  const uint64_t a01 = f2_pack(sa.x, sa.y), a23 = f2_pack(sa.z, sa.w);
+  const uint64_t b01 = f2_pack(sb.x, sb.y), b23 = f2_pack(sb.z, sb.w);
+  float a[4], b[4], u[4];
+  f2_unpack(a01, a[0], a[1]); f2_unpack(a23, a[2], a[3]);
+  f2_unpack(b01, b[0], b[1]); f2_unpack(b23, b[2], b[3]);
+  {
+    const uint64_t bt2 = f2_pack(bt, bt);
+    f2_unpack(f2_mul(bt2, f2_add(f2_pack(v4.x, v4.y), f2_pack(-a[0], -a[1]))), u[0], u[1]);
+    f2_unpack(f2_mul(bt2, f2_add(f2_pack(v4.z, v4.w), f2_pack(-a[2], -a[3]))), u[2], u[3]);
+  }
   if (rg == 0)
     store4(o_row + col, scale * fmaf(kq, u[0], b[0]), scale * fmaf(kq, u[1], b[1]),
            scale * fmaf(kq, u[2], b[2]), scale * fmaf(kq, u[3], b[3]));
