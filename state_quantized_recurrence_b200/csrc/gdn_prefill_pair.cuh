@@ -401,7 +401,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           const float *arow = sA + (r0 + rr) * LDT + c0b;
           const float *tcol = sT + c0b * LDT + c0b + cc;
           float4 p = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
+#pragma unroll 4
           for (int m = 0; m < 16; ++m) {
             const float a = arow[m];
             const float4 t4 = *reinterpret_cast<const float4 *>(tcol + m * LDT);
@@ -412,7 +412,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           const float *trow = sT + (r0 + rr) * LDT + r0;
           const float *pcol = sP + 16 * blk * LDT + cc;
           float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
+#pragma unroll 4
           for (int m = 0; m < 16; ++m) {
             const float t = trow[m];
             const float4 p4 = *reinterpret_cast<const float4 *>(pcol + m * LDT);
@@ -427,7 +427,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           const float *arow = sA + (32 + rr) * LDT;
           const float *tcol = sT + cc;
           float p[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
+#pragma unroll 4
           for (int m = 0; m < 32; ++m) {
             const float a = arow[m];
             const float4 t0v = *reinterpret_cast<const float4 *>(tcol + m * LDT);
@@ -441,7 +441,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           const float *trow = sT + (32 + rr) * LDT + 32;
           const float *pcol = sP + cc;
           float q[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
+#pragma unroll 4
           for (int m = 0; m < 32; ++m) {
             const float t = trow[m];
             const float4 p0v = *reinterpret_cast<const float4 *>(pcol + m * LDT);
