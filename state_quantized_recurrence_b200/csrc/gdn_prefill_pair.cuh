@@ -421,7 +421,11 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           *reinterpret_cast<float4 *>(sT + (r0 + rr) * LDT + c0b + cc) = make_float4(-q.x, -q.y, -q.z, -q.w);
         }
         asm volatile("bar.sync 3, 128;" ::: "memory");
-        // level 2: the lower-left 32x32 block: T_21 = -T_22 (A_21 T_11)
+        // level 2: the lower-left 32x32 block: T_21 = -T_22 (A_21 T_11).
+        // The products of levels 1 and 2 are unrolled by 4 only: fully
+        // unrolled, the producer's code grew large enough that instruction
+        // fetch, which neighbouring SMs share, slowed pairs by up to 20 %
+        // depending on where they ran
         {
           const int rr = tid >> 2, cc = (tid & 3) * 8;
           const float *arow = sA + (32 + rr) * LDT;
