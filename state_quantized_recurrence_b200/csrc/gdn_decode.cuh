@@ -250,31 +250,45 @@ struct StateIO {
 // are staged: decay, the key-axis reductions, the output, the delta update,
 // the QDQ and the store.  Shared by both decode kernels, so the fp32 and the
 // packed storage run the same arithmetic.
+// Key-indexed vectors (k, q, the per-key decay) are staged in shared memory
+// permuted, row r at (r % 16) * (d_k / 16) + r / 16, so that the d_k / 16
+// rows rg, rg + 16, ... of a thread are contiguous and arrive in 128-bit loads.
+template <int DK>
+__host__ __device__ constexpr int key_slot(int r) {
+  return (r % 16) * (DK / 16) + r / 16;
+}
+template <int RPT>
+__device__ __forceinline__ void load_rows(const float *s, int rg, float (&x)[RPT]) {
+#pragma unroll
+  for (int j = 0; j < RPT; j += 4) {
+    const float4 v = *reinterpret_cast<const float4 *>(s + rg * RPT + j);
+    x[j] = v.x; x[j + 1] = v.y; x[j + 2] = v.z; x[j + 3] = v.w;
+  }
+}
+
 template <typename Tin, int DK, int DV, bool PER_KEY, int QK, int GROUP, bool PACKED>
 __device__ __forceinline__ void decode_slab(float4 (&h)[DK / 16], const float *s_k,
                                             const float *s_q, const float *s_al, float a_scalar,
                                             float bt, float4 v4, float4 (*red_a)[16],
-                                            float4 (*red_b)[16], float *red_m, const StateRef &sr,
-                                            Tin *__restrict__ o_row, int col, float scale) {
+                                            float4 (*red_b)[16], float *red_m, float *s_kq,
+                                            const StateRef &sr, Tin *__restrict__ o_row, int col,
+                                            float scale) {
   using IO = StateIO<DK, DV, QK, GROUP, PACKED>;
   constexpr int RPT = IO::RPT;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int cq = tid & 15, rg = tid >> 4;
 
-  // k^T q, computed redundantly by every warp from shared memory.
-  float kq = 0.0f;
-#pragma unroll
-  for (int r = lane; r < DK; r += 32) kq += s_k[r] * s_q[r];
-  kq = warp_sum(kq);
-
   // Decay and the partial key-axis reductions a = Ht^T k, b = Ht^T q.
   // (fp32 pairs in packed f32x2 arithmetic: each lane rounds as the scalar
   // instruction)
+  float kv[RPT], qv[RPT], av[RPT];
+  load_rows<RPT>(s_k, rg, kv);
+  load_rows<RPT>(s_q, rg, qv);
+  if (PER_KEY) load_rows<RPT>(s_al, rg, av);
   uint64_t pa01 = 0, pa23 = 0, pb01 = 0, pb23 = 0;  // +0.0 pairs
 #pragma unroll
   for (int j = 0; j < RPT; ++j) {
-    const int r = rg + 16 * j;
-    const float al = PER_KEY ? s_al[r] : a_scalar, kr = s_k[r], qr = s_q[r];
+    const float al = PER_KEY ? av[j] : a_scalar, kr = kv[j], qr = qv[j];
     const uint64_t al2 = f2_pack(al, al), kr2 = f2_pack(kr, kr), qr2 = f2_pack(qr, qr);
     const uint64_t h01 = f2_mul(f2_pack(h[j].x, h[j].y), al2);
     const uint64_t h23 = f2_mul(f2_pack(h[j].z, h[j].w), al2);
@@ -298,7 +312,14 @@ __device__ __forceinline__ void decode_slab(float4 (&h)[DK / 16], const float *s
   __syncthreads();
   // the 8 warps' partial sums, in warp order (packed pairs, the scalar
   // additions' roundings), formed once per column by warp 0 (lanes 0-15: a,
-  // 16-31: b) into row 0 and read back by every thread
+  // 16-31: b) into row 0 and read back by every thread; warp 1 forms k^T q
+  if (warp == 1) {
+    float kq = 0.0f;
+#pragma unroll
+    for (int r = lane; r < DK; r += 32) kq += s_k[key_slot<DK>(r)] * s_q[key_slot<DK>(r)];
+    kq = warp_sum(kq);
+    if (lane == 0) *s_kq = kq;
+  }
   if (warp == 0) {
     float4(*red)[16] = lane < 16 ? red_a : red_b;
     const int c = lane & 15;
@@ -326,15 +347,18 @@ __device__ __forceinline__ void decode_slab(float4 (&h)[DK / 16], const float *s
     f2_unpack(f2_mul(bt2, f2_add(f2_pack(v4.x, v4.y), f2_pack(-a[0], -a[1]))), u[0], u[1]);
     f2_unpack(f2_mul(bt2, f2_add(f2_pack(v4.z, v4.w), f2_pack(-a[2], -a[3]))), u[2], u[3]);
   }
-  if (rg == 0)
+  if (rg == 0) {
+    const float kq = *s_kq;
     store4(o_row + col, scale * fmaf(kq, u[0], b[0]), scale * fmaf(kq, u[1], b[1]),
            scale * fmaf(kq, u[2], b[2]), scale * fmaf(kq, u[3], b[3]));
+  }
 
   // Delta update H = Ht + k u^T.
   const uint64_t u01 = f2_pack(u[0], u[1]), u23 = f2_pack(u[2], u[3]);
+  load_rows<RPT>(s_k, rg, kv);
 #pragma unroll
   for (int j = 0; j < RPT; ++j) {
-    const float kr = s_k[rg + 16 * j];
+    const float kr = kv[j];
     const uint64_t kr2 = f2_pack(kr, kr);
     f2_unpack(f2_fma(kr2, u01, f2_pack(h[j].x, h[j].y)), h[j].x, h[j].y);
     f2_unpack(f2_fma(kr2, u23, f2_pack(h[j].z, h[j].w)), h[j].z, h[j].w);
@@ -369,9 +393,13 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
               Tin *__restrict__ o, float scale) {
   using IO = StateIO<DK, DV, QK, GROUP, PACKED>;
   constexpr int NSC = QK == kQdqInt8 ? DK * (DV / GROUP) : DV / 64;  // scales per state
-  __shared__ float s_k[DK], s_q[DK], s_al[PER_KEY ? DK : 1];
+  // row-permuted (key_slot), 16-byte aligned for the 128-bit row loads
+  __shared__ __align__(16) float s_k[DK];
+  __shared__ __align__(16) float s_q[DK];
+  __shared__ __align__(16) float s_al[PER_KEY ? DK : 4];
   __shared__ float4 red_a[8][16], red_b[8][16];
   __shared__ float red_m[8];
+  __shared__ float s_kq;
 
   constexpr int nvt = DV / 64;
   const long long unit = blockIdx.x / nvt;  // sequence * H + head
@@ -385,16 +413,17 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
   IO::load(sr, rg, col, h);
 
   if (tid < DK) {
-    s_k[tid] = to_f32(k[unit * DK + tid]);
-    s_q[tid] = to_f32(q[unit * DK + tid]);
-    if (PER_KEY) s_al[tid] = expf(__ldg(g + unit * DK + tid));
+    s_k[key_slot<DK>(tid)] = to_f32(k[unit * DK + tid]);
+    s_q[key_slot<DK>(tid)] = to_f32(q[unit * DK + tid]);
+    if (PER_KEY) s_al[key_slot<DK>(tid)] = expf(__ldg(g + unit * DK + tid));
   }
   const float bt = __ldg(beta + unit);
   const float a_scalar = PER_KEY ? 0.0f : expf(__ldg(g + unit));
   const float4 v4 = load4(v + unit * DV + col);
   __syncthreads();
   decode_slab<Tin, DK, DV, PER_KEY, QK, GROUP, PACKED>(h, s_k, s_q, s_al, a_scalar, bt, v4, red_a,
-                                                       red_b, red_m, sr, o + unit * DV, col, scale);
+                                                       red_b, red_m, &s_kq, sr, o + unit * DV, col,
+                                                       scale);
 }
 
 // Conversion between the two storages of a state batch [n, d_k, d_v]: pack
