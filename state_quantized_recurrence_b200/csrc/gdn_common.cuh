@@ -153,18 +153,6 @@ __device__ __forceinline__ float2 qdq_fp8_2(float x0, float x1, const ScaleRecip
   return make_float2(__fmul_rn(c.x, sr.s), __fmul_rn(c.y, sr.s));
 }
 
-// The codes themselves (for packed state storage); the dequantized values
-// of the functions above are exactly code * s.
-// INT8 codes and QDQ values of four values (two packed quotients).
-__device__ __forceinline__ float4 int8_code4(float4 x, const ScaleRecip &sr) {
-  float4 q;
-  div_by_scale2(x.x, x.y, sr, q.x, q.y);
-  div_by_scale2(x.z, x.w, sr, q.z, q.w);
-  return make_float4(fminf(fmaxf(rintf(q.x), -127.0f), 127.0f),
-                     fminf(fmaxf(rintf(q.y), -127.0f), 127.0f),
-                     fminf(fmaxf(rintf(q.z), -127.0f), 127.0f),
-                     fminf(fmaxf(rintf(q.w), -127.0f), 127.0f));
-}
 __device__ __forceinline__ float4 mul4(float4 c, float s) {
   const uint64_t s2 = f2_pack(s, s);
   float4 y;
@@ -173,19 +161,13 @@ __device__ __forceinline__ float4 mul4(float4 c, float s) {
   return y;
 }
 
-// Integer-valued floats in [-2^22, 2^22] <-> their low byte / value through
-// the magic constant 1.5 * 2^23: adding it rounds to the nearest integer
-// (ties to even, the fp32 addition's own rounding) and leaves the integer in
-// the low mantissa bits, so neither direction needs a float <-> int
-// conversion instruction.
+// The packed state's codes: code * s is exactly the dequantized value of the
+// codecs above.  Integer-valued floats in [-2^22, 2^22] <-> their low byte /
+// value through the magic constant 1.5 * 2^23: adding it rounds to the
+// nearest integer (ties to even, the fp32 addition's own rounding) and leaves
+// the integer in the low mantissa bits, so neither direction needs a
+// float <-> int conversion instruction.
 constexpr float kMagicRound = 12582912.0f;  // 1.5 * 2^23
-// c = clamp(rint(q), -127, 127) as a float and as its two's-complement byte.
-__device__ __forceinline__ float int8_round_clamp(float q, uint32_t &byte) {
-  const float t = fminf(fmaxf(q, -127.0f), 127.0f) + kMagicRound;
-  byte = __float_as_uint(t) & 0xffu;
-  return t - kMagicRound;
-}
-
 // The four INT8 codes in the bytes of w (two's complement), exactly, as
 // floats: flipping each byte's sign bit gives u = c + 128 in 0 .. 255, prmt
 // puts u under the upper bytes of 1.5 * 2^23 (the float 1.5 * 2^23 + u, an
@@ -226,14 +208,6 @@ __device__ __forceinline__ uint32_t int8_round4(uint64_t q01, uint64_t q23, floa
   return w;
 }
 
-__device__ __forceinline__ float int8_code(float x, const ScaleRecip &sr) {
-  return fminf(fmaxf(rintf(div_by_scale(x, sr)), -127.0f), 127.0f);
-}
-// E4M3 bytes of x0 / s and x1 / s (x0 in the low byte).
-__device__ __forceinline__ unsigned short e4m3_code2(float x0, float x1, const ScaleRecip &sr) {
-  return (unsigned short)__nv_cvt_float2_to_fp8x2(make_float2(div_by_scale(x0, sr), div_by_scale(x1, sr)),
-                                                  __NV_SATFINITE, __NV_E4M3);
-}
 // Two E4M3 bytes (low byte first) -> their values, exactly.
 __device__ __forceinline__ float2 e4m3_pair_to_f2(unsigned short p) {
   __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)p, __NV_E4M3);
