@@ -237,28 +237,34 @@ def cpu_model() -> str:
     return "unknown"
 
 
-def cpu_baseline_prefill(case, inp, max_seconds: float = 12.0) -> dict:
+def cpu_baseline_prefill(case, inp, min_seconds: float = 8.0, max_passes: int = 50) -> dict:
     """The oracle as it stands, on whole sequences of the workload (all
-    heads), on this host's cores; tokens/s scaled from the sample.  One
-    sequence is also run on a single thread."""
+    heads), on this host's cores; tokens/s over passes through the
+    workload's sequences until about `min_seconds` of CPU work (a whole
+    sequence at a time).  One sequence is also run on a single thread."""
     import oracle
     threads = len(os.sched_getaffinity(0))
     lengths = [int(x) for x in inp["lengths"]]
     packed = inp["cu_seqlens"] is not None
-    done, tokens, t_total, start = 0, 0, 0.0, 0
-    for s, n in enumerate(lengths):
-        # one whole sequence (all heads): a batch row, or its packed token range
-        sl = (slice(0, 1), slice(start, start + n)) if packed else (slice(s, s + 1),)
-        st_in = inp["state_in"][s:s + 1] if inp["state_in"] is not None else None
-        t0 = time.perf_counter()
-        oracle.recurrence(inp["q"][sl], inp["k"][sl], inp["v"][sl], inp["g"][sl],
-                          inp["beta"][sl], st_in, oracle.dense_cu_seqlens(1, n),
-                          per_key_gate=case.gate == "per_key", qdq=case.qdq, n_threads=threads)
-        t_total += time.perf_counter() - t0
-        start += n
-        done += 1
-        tokens += n
-        if t_total * (done + 1) / done > max_seconds:
+    done, tokens, t_total = 0, 0, 0.0
+    for _ in range(max_passes):
+        start = 0
+        for s, n in enumerate(lengths):
+            # one whole sequence (all heads): a batch row, or its packed token range
+            sl = (slice(0, 1), slice(start, start + n)) if packed else (slice(s, s + 1),)
+            st_in = inp["state_in"][s:s + 1] if inp["state_in"] is not None else None
+            t0 = time.perf_counter()
+            oracle.recurrence(inp["q"][sl], inp["k"][sl], inp["v"][sl], inp["g"][sl],
+                              inp["beta"][sl], st_in, oracle.dense_cu_seqlens(1, n),
+                              per_key_gate=case.gate == "per_key", qdq=case.qdq,
+                              n_threads=threads)
+            t_total += time.perf_counter() - t0
+            start += n
+            done += 1
+            tokens += n
+            if t_total >= min_seconds:
+                break
+        if t_total >= min_seconds:
             break
     # the first sequence again on one thread (its first 1024 tokens at most)
     n1 = min(1024, lengths[0])
@@ -270,25 +276,40 @@ def cpu_baseline_prefill(case, inp, max_seconds: float = 12.0) -> dict:
                       per_key_gate=case.gate == "per_key", qdq=case.qdq, n_threads=1)
     t1 = time.perf_counter() - t0
     return {"value": tokens / t_total, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-            "sample": f"{done} of {len(lengths)} sequences ({tokens} tokens x {case.H} heads), "
-                      f"fp64 token recurrence + fp32 {case.qdq} codec, OpenMP over heads",
+            "sample": f"{done} whole sequences of the workload's {len(lengths)}, cycling "
+                      f"({tokens} tokens x {case.H} heads), fp64 token recurrence + fp32 "
+                      f"{case.qdq} codec, OpenMP over heads",
             "seconds": round(t_total, 3), "value_1_thread": round(n1 / t1, 1),
             "sample_1_thread": f"{n1} tokens x {case.H} heads of sequence 0",
             "cpu_model": cpu_model()}
 
 
-def cpu_baseline_decode(case, inp, state) -> dict:
+def cpu_baseline_decode(case, inp, state, min_seconds: float = 6.0) -> dict:
+    """The decode oracle on all sequences of the workload: one token first,
+    then as many further tokens as about `min_seconds` of CPU work allow."""
     import oracle
     threads = len(os.sched_getaffinity(0))
-    n_seq = 64
-    sl = (slice(0, 1), slice(0, n_seq))
-    t0 = time.perf_counter()
-    oracle.decode(inp["dec_q"][sl], inp["dec_k"][sl], inp["dec_v"][sl], inp["dec_g"][sl],
-                  inp["dec_beta"][sl], state[:n_seq], per_key_gate=False, qdq=case.qdq,
-                  n_threads=threads)
-    dt = time.perf_counter() - t0
-    return {"value": n_seq * case.H / dt, "unit": "updates/s", "cores": threads, "kind": "oracle",
-            "sample": f"1 token of {n_seq} of {case.n_seq} sequences x {case.H} heads",
+    n_seq = case.n_seq
+
+    def run(t0_tok, n_tok, st):
+        sl = (slice(t0_tok, t0_tok + n_tok), slice(0, n_seq))
+        t0 = time.perf_counter()
+        res = oracle.decode(inp["dec_q"][sl], inp["dec_k"][sl], inp["dec_v"][sl],
+                            inp["dec_g"][sl], inp["dec_beta"][sl], st, per_key_gate=False,
+                            qdq=case.qdq, n_threads=threads)
+        return time.perf_counter() - t0, res[1]
+
+    dt, st = run(0, 1, state[:n_seq])
+    steps = int(inp["dec_q"].shape[0])
+    more = max(0, min(steps - 1, int((min_seconds - dt) / max(dt, 1e-6))))
+    n_tok = 1
+    if more > 0:
+        dt2, _ = run(1, more, st)
+        dt += dt2
+        n_tok += more
+    return {"value": n_tok * n_seq * case.H / dt, "unit": "updates/s", "cores": threads,
+            "kind": "oracle",
+            "sample": f"{n_tok} tokens of all {n_seq} sequences x {case.H} heads",
             "seconds": round(dt, 3)}
 
 
@@ -440,7 +461,7 @@ def measure_prefill(args, dist, dev, stream, sampler, peaks, case, steps, warmup
         "clocks": sampler.summary(t_wall0, t_wall1),
     }
     if cpu and dist.rank == 0 and not args.no_cpu_baseline:
-        res["cpu_baseline"] = cpu_baseline_prefill(case, inp, max_seconds=8.0)
+        res["cpu_baseline"] = cpu_baseline_prefill(case, inp, min_seconds=4.0)
     if keep:
         return res, (inp, d, o, st, step, tokens, nbytes)
     del d, o, st
