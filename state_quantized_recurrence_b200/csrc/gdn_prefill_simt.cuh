@@ -64,6 +64,12 @@ __device__ __forceinline__ float dot4(float4 a, float4 b) {
   return a.x * b.x + a.y * b.y + a.z * b.z + a.w * b.w;
 }
 
+// The products below run as packed f32x2 FMAs (two lanes per instruction,
+// each rounded as the scalar FMA): the kernel is bound by instruction issue.
+__device__ __forceinline__ uint64_t lo2(float4 v) { return f2_pack(v.x, v.y); }
+__device__ __forceinline__ uint64_t hi2(float4 v) { return f2_pack(v.z, v.w); }
+__device__ __forceinline__ uint64_t bc2(float x) { return f2_pack(x, x); }
+
 // C = M1 M2 for lower-triangular 64 x 64 operands (row stride LDT), the 4 x 4
 // block (rows 4 R .., columns 4 C ..) of this thread into `acc` (zero above
 // the diagonal): terms with i outside [4 C, 4 R + 3] vanish because the
@@ -244,11 +250,13 @@ prefill_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
 
     // ---- P3: A = strict_lower(diag(b) Kp Km^T), Aqk = lower(Qp Km^T) ----
     {
-      float accA[4][4], accQ[4][4];
+      // each dot product as two packed partial sums (even / odd keys),
+      // folded at the end
+      uint64_t pA[4][4], pQ[4][4];
 #pragma unroll
       for (int m = 0; m < 4; ++m)
 #pragma unroll
-        for (int mm = 0; mm < 4; ++mm) accA[m][mm] = accQ[m][mm] = 0.0f;
+        for (int mm = 0; mm < 4; ++mm) pA[m][mm] = pQ[m][mm] = 0ull;
       for (int c = 0; c < DK; c += 4) {
         float4 kp[4], qp[4], km[4];
 #pragma unroll
@@ -261,10 +269,21 @@ prefill_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
         for (int m = 0; m < 4; ++m)
 #pragma unroll
           for (int mm = 0; mm < 4; ++mm) {
-            accA[m][mm] += dot4(kp[m], km[mm]);
-            accQ[m][mm] += dot4(qp[m], km[mm]);
+            pA[m][mm] = f2_fma(hi2(kp[m]), hi2(km[mm]), f2_fma(lo2(kp[m]), lo2(km[mm]), pA[m][mm]));
+            pQ[m][mm] = f2_fma(hi2(qp[m]), hi2(km[mm]), f2_fma(lo2(qp[m]), lo2(km[mm]), pQ[m][mm]));
           }
       }
+      float accA[4][4], accQ[4][4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+#pragma unroll
+        for (int mm = 0; mm < 4; ++mm) {
+          float a0, a1, q0, q1;
+          f2_unpack(pA[m][mm], a0, a1);
+          f2_unpack(pQ[m][mm], q0, q1);
+          accA[m][mm] = a0 + a1;
+          accQ[m][mm] = q0 + q1;
+        }
       __syncthreads();  // the gate cumsum in sR is consumed; A/Aqk overwrite it
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
@@ -401,6 +420,12 @@ prefill_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
         float4 u4 = *reinterpret_cast<float4 *>(sV + (rb + 16 * m) * LDV + 4 * cb);
         acc[m][0] = u4.x; acc[m][1] = u4.y; acc[m][2] = u4.z; acc[m][3] = u4.w;
       }
+      uint64_t a01[4], a23[4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        a01[m] = f2_pack(acc[m][0], acc[m][1]);
+        a23[m] = f2_pack(acc[m][2], acc[m][3]);
+      }
       for (int c = 0; c < DK; c += 4) {
         float4 hh[4];
 #pragma unroll
@@ -411,10 +436,16 @@ prefill_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
           const float we[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            acc[m][0] -= we[e] * hh[e].x; acc[m][1] -= we[e] * hh[e].y;
-            acc[m][2] -= we[e] * hh[e].z; acc[m][3] -= we[e] * hh[e].w;
+            const uint64_t nw = bc2(-we[e]);
+            a01[m] = f2_fma(nw, lo2(hh[e]), a01[m]);
+            a23[m] = f2_fma(nw, hi2(hh[e]), a23[m]);
           }
         }
+      }
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        f2_unpack(a01[m], acc[m][0], acc[m][1]);
+        f2_unpack(a23[m], acc[m][2], acc[m][3]);
       }
 #pragma unroll
       for (int m = 0; m < 4; ++m)
@@ -426,10 +457,9 @@ prefill_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
     // ---- P7: O = scale ((Q e^G) H0 + Aqk Vn) ----
     {
       float acc[4][4];
+      uint64_t a01[4], a23[4];
 #pragma unroll
-      for (int m = 0; m < 4; ++m)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[m][e] = 0.0f;
+      for (int m = 0; m < 4; ++m) a01[m] = a23[m] = 0ull;
       for (int c = 0; c < DK; c += 4) {
         float4 hh[4];
 #pragma unroll
@@ -440,8 +470,9 @@ prefill_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
           const float qe[4] = {qq.x, qq.y, qq.z, qq.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            acc[m][0] += qe[e] * hh[e].x; acc[m][1] += qe[e] * hh[e].y;
-            acc[m][2] += qe[e] * hh[e].z; acc[m][3] += qe[e] * hh[e].w;
+            const uint64_t q2 = bc2(qe[e]);
+            a01[m] = f2_fma(q2, lo2(hh[e]), a01[m]);
+            a23[m] = f2_fma(q2, hi2(hh[e]), a23[m]);
           }
         }
       }
@@ -451,9 +482,15 @@ prefill_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
           float2 aa = *reinterpret_cast<float2 *>(sAqk + (rb + 16 * m) * LDA + i);
-          acc[m][0] += aa.x * v0.x + aa.y * v1.x; acc[m][1] += aa.x * v0.y + aa.y * v1.y;
-          acc[m][2] += aa.x * v0.z + aa.y * v1.z; acc[m][3] += aa.x * v0.w + aa.y * v1.w;
+          const uint64_t x2 = bc2(aa.x), y2 = bc2(aa.y);
+          a01[m] = f2_fma(y2, lo2(v1), f2_fma(x2, lo2(v0), a01[m]));
+          a23[m] = f2_fma(y2, hi2(v1), f2_fma(x2, hi2(v0), a23[m]));
         }
+      }
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        f2_unpack(a01[m], acc[m][0], acc[m][1]);
+        f2_unpack(a23[m], acc[m][2], acc[m][3]);
       }
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
@@ -476,18 +513,31 @@ prefill_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
         const float en = sEn[r];
         acc[j][0] = en * h0.x; acc[j][1] = en * h0.y; acc[j][2] = en * h0.z; acc[j][3] = en * h0.w;
       }
+      uint64_t a01[RPT], a23[RPT];
+#pragma unroll
+      for (int j = 0; j < RPT; ++j) {
+        a01[j] = f2_pack(acc[j][0], acc[j][1]);
+        a23[j] = f2_pack(acc[j][2], acc[j][3]);
+      }
       for (int i = 0; i < 64; ++i) {
         float4 vn = *reinterpret_cast<float4 *>(sV + i * LDV + 4 * cb);
+        const uint64_t v01 = lo2(vn), v23 = hi2(vn);
 #pragma unroll
         for (int j4 = 0; j4 < RPT; j4 += 4) {
           float4 kc = *reinterpret_cast<float4 *>(sX + i * LDK + rb * RPT + j4);
           const float ke[4] = {kc.x, kc.y, kc.z, kc.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            acc[j4 + e][0] += ke[e] * vn.x; acc[j4 + e][1] += ke[e] * vn.y;
-            acc[j4 + e][2] += ke[e] * vn.z; acc[j4 + e][3] += ke[e] * vn.w;
+            const uint64_t k2 = bc2(ke[e]);
+            a01[j4 + e] = f2_fma(k2, v01, a01[j4 + e]);
+            a23[j4 + e] = f2_fma(k2, v23, a23[j4 + e]);
           }
         }
+      }
+#pragma unroll
+      for (int j = 0; j < RPT; ++j) {
+        f2_unpack(a01[j], acc[j][0], acc[j][1]);
+        f2_unpack(a23[j], acc[j][2], acc[j][3]);
       }
       if (qdq_kind == kQdqInt8) {
 #pragma unroll
