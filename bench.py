@@ -498,6 +498,16 @@ def run_ours(args, dist: Dist) -> dict:
         dist.close()
         return {"metric": dec["metric"], "value": dec["value"], "unit": dec["unit"],
                 "n_gpus": dist.world, "impl": "ours", "decode": dec}
+    if args.only == "kda":  # profiler captures of the CUDA-core prefill kernel
+        kcase = gs.small_case("kda_prefill", decode_steps=0)
+        if args.small:  # the same 128 CTAs, 8 chunks each
+            kcase = gs.small_case("kda_prefill", T=512, decode_steps=0)
+        kda = measure_prefill(args, dist, dev, stream, sampler, peaks, kcase, args.steps,
+                              args.warmup)
+        sampler.stop()
+        dist.close()
+        return {"metric": "prefill tokens/s", "value": kda["value"], "unit": kda["unit"],
+                "n_gpus": dist.world, "impl": "ours", "kda_prefill": kda}
 
     # ---------------- prefill (headline) ----------------
     case = gs.CONFIGS["gdn_prefill"]
@@ -760,7 +770,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-decode", action="store_true")
-    ap.add_argument("--only", choices=["prefill", "decode", "decode_packed", "backward"],
+    ap.add_argument("--only", choices=["prefill", "decode", "decode_packed", "backward", "kda"],
                     default=None,
                     help="measure one kernel only (profiler captures)")
     ap.add_argument("--no-e2e", action="store_true")

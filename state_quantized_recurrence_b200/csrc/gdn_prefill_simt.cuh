@@ -81,6 +81,7 @@ __device__ __forceinline__ void lower_mul_block(const float *M1, const float *M2
 #pragma unroll
     for (int b = 0; b < 4; ++b) acc[a][b] = 0.0f;
   if (C > R) return;
+  uint64_t a01[4] = {0ull, 0ull, 0ull, 0ull}, a23[4] = {0ull, 0ull, 0ull, 0ull};
   for (int i0 = 4 * C; i0 <= 4 * R; i0 += 4) {
     float4 m2[4];
 #pragma unroll
@@ -91,10 +92,15 @@ __device__ __forceinline__ void lower_mul_block(const float *M1, const float *M2
       const float w[4] = {m1.x, m1.y, m1.z, m1.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        acc[a][0] += w[e] * m2[e].x; acc[a][1] += w[e] * m2[e].y;
-        acc[a][2] += w[e] * m2[e].z; acc[a][3] += w[e] * m2[e].w;
+        a01[a] = f2_fma(bc2(w[e]), lo2(m2[e]), a01[a]);
+        a23[a] = f2_fma(bc2(w[e]), hi2(m2[e]), a23[a]);
       }
     }
+  }
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    f2_unpack(a01[a], acc[a][0], acc[a][1]);
+    f2_unpack(a23[a], acc[a][2], acc[a][3]);
   }
 }
 
@@ -392,14 +398,18 @@ prefill_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
 #pragma unroll
         for (int r = 0; r < kChunk; ++r) {
           if (r < n) {
-            float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
+            // partial sums (p0, p1) and (p2, p3) as packed pairs
+            uint64_t p01 = 0ull, p23 = 0ull;
             const float *arow = sA + r * LDA;
 #pragma unroll
             for (int i = 0; i + 1 < r; i += 2) {
-              float2 aa = *reinterpret_cast<const float2 *>(arow + i);
-              if (i & 2) { p2 += aa.x * x[i]; p3 += aa.y * x[i + 1]; }
-              else       { p0 += aa.x * x[i]; p1 += aa.y * x[i + 1]; }
+              const uint64_t aa = *reinterpret_cast<const uint64_t *>(arow + i);
+              if (i & 2) p23 = f2_fma(aa, f2_pack(x[i], x[i + 1]), p23);
+              else       p01 = f2_fma(aa, f2_pack(x[i], x[i + 1]), p01);
             }
+            float p0, p1, p2, p3;
+            f2_unpack(p01, p0, p1);
+            f2_unpack(p23, p2, p3);
             if (r & 1) p0 += arow[r - 1] * x[r - 1];
             const float xr = colp[r * ld] - ((p0 + p1) + (p2 + p3));
             x[r] = xr;
