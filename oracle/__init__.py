@@ -25,6 +25,7 @@ and requires each to fail a pin.  Nothing stored or computed here comes from the
 from __future__ import annotations
 
 import ctypes
+import hashlib
 import os
 import subprocess
 from typing import Optional
@@ -47,14 +48,22 @@ CHUNK = 64
 def build(force: bool = False, src: str = _SRC, out: str = _LIB) -> str:
     """Compile ``liboracle.so`` with gcc (no fast-math, no FP contraction).
     ``src``/``out`` let the tests compile a copy with a planted mistake."""
-    if (not force and os.path.exists(out)
-            and os.path.getmtime(out) >= os.path.getmtime(src)):
-        return out
     cmd = ["gcc", "-std=c11", "-O2", "-fPIC", "-shared", "-fopenmp",
            "-fno-fast-math", "-ffp-contract=off", "-fno-finite-math-only",
            "-o", out + ".tmp", src, "-lm"]
+    # staleness by content (flags + source), not modification times
+    h = hashlib.sha256(" ".join(cmd[:-4]).encode())
+    with open(src, "rb") as f:
+        h.update(f.read())
+    digest, stamp = h.hexdigest(), out + ".sha256"
+    if not force and os.path.exists(out) and os.path.exists(stamp):
+        with open(stamp) as f:
+            if f.read().strip() == digest:
+                return out
     subprocess.run(cmd, check=True)
     os.replace(out + ".tmp", out)
+    with open(stamp, "w") as f:
+        f.write(digest + "\n")
     return out
 
 

@@ -9,6 +9,7 @@ file so that it travels with the source tree.
 from __future__ import annotations
 
 import glob
+import hashlib
 import os
 import subprocess
 import sys
@@ -38,22 +39,40 @@ def _sources():
                   + glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
+STAMP = LIB + ".sha256"
+
+
+def source_digest() -> str:
+    """Hash of the compiler flags and every source's name and contents.
+    Staleness is decided by content, not modification times, which a copy
+    of the tree to another machine need not preserve."""
+    h = hashlib.sha256(" ".join(NVCC_FLAGS).encode())
+    for s in _sources():
+        h.update(os.path.relpath(s, ROOT).encode())
+        with open(s, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+    if not (os.path.exists(LIB) and os.path.exists(STAMP)):
         return False
-    t = os.path.getmtime(LIB)
-    return all(os.path.getmtime(s) <= t for s in _sources())
+    with open(STAMP) as f:
+        return f.read().strip() == source_digest()
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
     if not force and up_to_date():
         return LIB
+    digest = source_digest()
     tmp = LIB + ".tmp"
     cmd = [_nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-o", tmp, MAIN]
     if verbose:
         print(" ".join(cmd), flush=True)
     subprocess.run(cmd, check=True)
     os.replace(tmp, LIB)
+    with open(STAMP, "w") as f:
+        f.write(digest + "\n")
     return LIB
 
 
