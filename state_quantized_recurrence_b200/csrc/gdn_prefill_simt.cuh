@@ -453,7 +453,9 @@ prefill_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
     }
     __syncthreads();
 
-    // ---- P6: Vn = U - W H0 (in place in sV) ----
+    // ---- P6: Vn = U - W H0 (in place in sV), and in the same pass over H0
+    //      the outputs' first term (Q e^G) H0, kept packed in o01 / o23 ----
+    uint64_t o01[4], o23[4];
     {
       float acc[4][4];
 #pragma unroll
@@ -466,6 +468,7 @@ prefill_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
       for (int m = 0; m < 4; ++m) {
         a01[m] = f2_pack(acc[m][0], acc[m][1]);
         a23[m] = f2_pack(acc[m][2], acc[m][3]);
+        o01[m] = o23[m] = 0ull;
       }
       for (int c = 0; c < DK; c += 4) {
         float4 hh[4];
@@ -474,12 +477,16 @@ prefill_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
           float4 w = *reinterpret_cast<float4 *>(sK + (rb + 16 * m) * LDK + c);
+          float4 qq = *reinterpret_cast<float4 *>(sQ + (rb + 16 * m) * LDK + c);
           const float we[4] = {w.x, w.y, w.z, w.w};
+          const float qe[4] = {qq.x, qq.y, qq.z, qq.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const uint64_t nw = bc2(-we[e]);
+            const uint64_t nw = bc2(-we[e]), q2 = bc2(qe[e]);
             a01[m] = f2_fma(nw, lo2(hh[e]), a01[m]);
             a23[m] = f2_fma(nw, hi2(hh[e]), a23[m]);
+            o01[m] = f2_fma(q2, lo2(hh[e]), o01[m]);
+            o23[m] = f2_fma(q2, hi2(hh[e]), o23[m]);
           }
         }
       }
@@ -495,28 +502,10 @@ prefill_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
     }
     __syncthreads();
 
-    // ---- P7: O = scale ((Q e^G) H0 + Aqk Vn) ----
+    // ---- P7: O = scale ((Q e^G) H0 + Aqk Vn), the first term from P6 ----
     {
       float acc[4][4];
-      uint64_t a01[4], a23[4];
-#pragma unroll
-      for (int m = 0; m < 4; ++m) a01[m] = a23[m] = 0ull;
-      for (int c = 0; c < DK; c += 4) {
-        float4 hh[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) hh[e] = *reinterpret_cast<float4 *>(sH + (c + e) * LDV + 4 * cb);
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          float4 qq = *reinterpret_cast<float4 *>(sQ + (rb + 16 * m) * LDK + c);
-          const float qe[4] = {qq.x, qq.y, qq.z, qq.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const uint64_t q2 = bc2(qe[e]);
-            a01[m] = f2_fma(q2, lo2(hh[e]), a01[m]);
-            a23[m] = f2_fma(q2, hi2(hh[e]), a23[m]);
-          }
-        }
-      }
+      uint64_t *a01 = o01, *a23 = o23;
       for (int i = 0; i < 64; i += 2) {
         float4 v0 = *reinterpret_cast<float4 *>(sV + i * LDV + 4 * cb);
         float4 v1 = *reinterpret_cast<float4 *>(sV + (i + 1) * LDV + 4 * cb);
