@@ -13,7 +13,9 @@ Modes:
   numpy, used to pin the chunked algebra against the token recurrence (and,
   with ``solve=("neumann", d)``, the approximate solve).
 * :func:`oracle.backward.backward` - the fp64 reverse pass of the token
-  recurrence with the state QDQ passed straight through.
+  recurrence with the state QDQ passed straight through;
+  :func:`oracle.backward.chunked_backward` - the same gradients chunk by
+  chunk (the adjoint of the chunked WY form), pinned to the token pass.
 
 Pins: every function here is checked by ``tests/test_oracle_*.py`` against
 closed forms, invariants, special cases and library routines (see the

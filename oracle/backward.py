@@ -28,7 +28,8 @@ Reverse, with dH the gradient of the loss with respect to H_t (at the end:
 Pins (tests/test_oracle_backward.py): central finite differences of the C
 token recurrence with QDQ off; with QDQ on, finite differences of the forward
 whose QDQ residuals QDQ(Hn) - Hn are frozen at their unperturbed values (its
-exact derivative is the straight-through gradient); closed forms.
+exact derivative is the straight-through gradient); closed forms.  The
+chunk-level pass at the end of this file is pinned to the token pass.
 """
 
 from __future__ import annotations
@@ -153,4 +154,139 @@ def backward(q, k, v, g, beta, state_in, cu_seqlens, do, dstate_out, *,
                     dg[tok, h] = al[0] * dal.sum()
                 dH = al[:, None] * dHt
             dst[s, h] = dH
+    return dq, dk, dv, dg, dbeta, dst
+
+
+# ----------------------------------------------------------------------------
+# Chunk-level reverse pass
+#
+# The adjoint of the chunked WY form (:func:`oracle.chunked.chunk_step`), one
+# 64-token chunk at a time from the chunk-start states of the forward: the
+# shape a chunked kernel computes.  The pages fix only the forward steps and
+# the straight-through QDQ; this is the exact derivative of those steps,
+# taken through each product in reverse order, and its pin is equality with
+# :func:`backward` (itself pinned by finite differences).  With G the
+# within-chunk cumulative log gate ([n, d_k]; a scalar gate broadcast over
+# the keys), D[r, i, c] = exp(G[r, c] - G[i, c]), gamma = exp(G),
+# E = exp(G[n-1] - G), and the forward's A, T, W, U, V_new, A_qk:
+#
+#   dV_new = scale A_qk^T dO + (K * E) dH_n
+#   dH_0   = scale (Q * gamma)^T dO + diag(gamma_n) dH_n - W^T dV_new
+#   dA_qk  = lower(scale dO V_new^T),       dU = dV_new,  dW = -dV_new H_0^T
+#   dT     = dW (beta K gamma)^T + dU (beta V)^T
+#   dA     = strict_lower(-T^T dT T^T)
+#
+# then the products A = strict_lower(beta K K^T * D), A_qk = lower(Q K^T * D),
+# W = T beta (K * gamma), U = T beta V, O and H_n give dq, dk, dv, dbeta and
+# dG, and dg_t = sum_{r >= t} dG_r (summed over the keys for a scalar gate).
+# ----------------------------------------------------------------------------
+
+def chunk_backward_step(Q, K, V, g, beta, H0, dO, dHn, *, scale: float):
+    """Reverse of one chunk (per-key gate form, fp64).  ``g`` is [n, d_k]
+    (broadcast a scalar gate before the call).  Returns
+    ``dQ, dK, dV, dg [n, d_k], dbeta [n], dH0``."""
+    n, d_k = K.shape
+    G = np.cumsum(g, axis=0)
+    gamma = np.exp(G)
+    D = np.exp(G[:, None, :] - G[None, :, :])          # [n, n, d_k]
+    E = np.exp(G[n - 1][None, :] - G)                   # [n, d_k]
+    low_strict = np.tril(np.ones((n, n)), k=-1)
+    low = np.tril(np.ones((n, n)))
+    # forward quantities
+    KK = np.einsum("rc,ic,ric->ri", K, K, D)
+    A = low_strict * (beta[:, None] * KK)
+    T = np.linalg.inv(np.eye(n) + A)
+    BKg = beta[:, None] * (K * gamma)
+    BV = beta[:, None] * V
+    W = T @ BKg
+    U = T @ BV
+    Vn = U - W @ H0
+    QK = np.einsum("rc,ic,ric->ri", Q, K, D)
+    Aqk = low * QK
+    # outputs and the state
+    dVn = scale * (Aqk.T @ dO) + (K * E) @ dHn
+    dH0 = scale * ((Q * gamma).T @ dO) + gamma[n - 1][:, None] * dHn - W.T @ dVn
+    dAqk = low * (scale * (dO @ Vn.T))
+    dQg = scale * (dO @ H0.T)                           # d(Q * gamma)
+    dKe = Vn @ dHn.T                                    # d(K * E)
+    dQ = dQg * gamma
+    dK = dKe * E
+    dgam = dQg * Q
+    dG = np.zeros_like(G)
+    dEK = dKe * K * E                                   # d/dG of E terms
+    dG -= dEK
+    dG[n - 1] += dEK.sum(axis=0)
+    dG[n - 1] += np.sum(H0 * dHn, axis=1) * gamma[n - 1]
+    # V_new = U - W H0
+    dU = dVn
+    dW = -dVn @ H0.T
+    # W = T (beta K gamma), U = T (beta V)
+    dT = dW @ BKg.T + dU @ BV.T
+    dBKg = T.T @ dW
+    dBV = T.T @ dU
+    dbeta = np.sum(dBKg * K * gamma, axis=1) + np.sum(dBV * V, axis=1)
+    dK += beta[:, None] * dBKg * gamma
+    dgam += beta[:, None] * dBKg * K
+    dV = beta[:, None] * dBV
+    # T = (I + A)^-1
+    dA = low_strict * (-(T.T @ dT @ T.T))
+    # A = strict_lower(beta K K^T * D)
+    dbeta += np.sum(dA * KK, axis=1)
+    dKK = beta[:, None] * dA
+    dK += np.einsum("ri,ic,ric->rc", dKK, K, D) + np.einsum("ri,rc,ric->ic", dKK, K, D)
+    dD = np.einsum("ri,rc,ic->ric", dKK, K, K)
+    # A_qk = lower(Q K^T * D)
+    dQ += np.einsum("ri,ic,ric->rc", dAqk, K, D)
+    dK += np.einsum("ri,rc,ric->ic", dAqk, Q, D)
+    dD += np.einsum("ri,rc,ic->ric", dAqk, Q, K)
+    # D[r, i] = exp(G_r - G_i), gamma = exp(G)
+    dDD = dD * D
+    dG += dDD.sum(axis=1) - dDD.sum(axis=0)
+    dG += dgam * gamma
+    # G = cumsum(g)
+    dg = np.cumsum(dG[::-1], axis=0)[::-1]
+    return dQ, dK, dV, dg, dbeta, dH0
+
+
+def chunked_backward(q, k, v, g, beta, state_in, cu_seqlens, do, dstate_out, *,
+                     per_key_gate: bool, qdq: str = "none", chunk: int = CHUNK,
+                     record: bool = False):
+    """Chunk-level reverse pass, same arguments and returns as
+    :func:`backward` (QDQ at every chunk end, passed straight through).  The
+    chunk-start states come from the token forward.  With ``record`` also
+    returns ``{(s, h, c): dH}``, the gradient with respect to each chunk's
+    end state."""
+    _, _, _, states = forward(q, k, v, g, beta, state_in, cu_seqlens,
+                              per_key_gate=per_key_gate, qdq=qdq,
+                              boundary_every=chunk, record=True)
+    q, k, v, g, beta, st, cu = _prep(q, k, v, g, beta, state_in, cu_seqlens, per_key_gate)
+    n_seq, H, d_k, d_v = st.shape
+    scale = 1.0 / np.sqrt(d_k)
+    do = _f64(do).reshape(-1, H, d_v)
+    dso = (np.zeros_like(st) if dstate_out is None
+           else _f64(dstate_out).reshape(n_seq, H, d_k, d_v))
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    dg, dbeta = np.zeros_like(g), np.zeros_like(beta)
+    dst = np.zeros_like(st)
+    dH_end = {}
+    for s in range(n_seq):
+        for h in range(H):
+            dH = dso[s, h].copy()
+            t0, L = int(cu[s]), int(cu[s + 1] - cu[s])
+            starts = list(range(0, L, chunk))
+            for ci in range(len(starts) - 1, -1, -1):
+                c0 = starts[ci]
+                c1 = min(c0 + chunk, L)
+                a, b = t0 + c0, t0 + c1
+                gc = g[a:b, h] if per_key_gate else g[a:b, h][:, None] * np.ones((1, d_k))
+                dH_end[(s, h, ci)] = dH.copy()
+                dQ, dK, dV, dgc, dbc, dH = chunk_backward_step(
+                    q[a:b, h], k[a:b, h], v[a:b, h], gc, beta[a:b, h],
+                    states[(s, h, c0)], do[a:b, h], dH, scale=scale)
+                dq[a:b, h], dk[a:b, h], dv[a:b, h] = dQ, dK, dV
+                dg[a:b, h] = dgc if per_key_gate else dgc.sum(axis=1)
+                dbeta[a:b, h] = dbc
+            dst[s, h] = dH
+    if record:
+        return dq, dk, dv, dg, dbeta, dst, dH_end
     return dq, dk, dv, dg, dbeta, dst

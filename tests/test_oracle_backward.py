@@ -6,7 +6,9 @@
 * QDQ on: finite differences of the forward whose QDQ residuals are frozen at
   their unperturbed values (so its exact derivative is the straight-through
   gradient) match the backward's gradients;
-* closed forms at beta = 0, g = 0 (the state stays H0).
+* closed forms at beta = 0, g = 0 (the state stays H0);
+* the chunk-level reverse pass (the adjoint of the chunked WY form, chunk by
+  chunk from the forward's chunk-start states) equals the token reverse pass.
 """
 
 import numpy as np
@@ -118,3 +120,28 @@ def test_backward_closed_forms_constant_state():
         np.testing.assert_allclose(dg[t, 0], np.sum(H0 * dHn), rtol=0, atol=1e-12)
         np.testing.assert_allclose(dbeta[t, 0], (dHn.T @ k[t]) @ (v[t] - H0.T @ k[t]),
                                    rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("per_key", [False, True])
+@pytest.mark.parametrize("mode", ["none", "int8_g32", "fp8_tile64"])
+def test_chunked_backward_matches_token_backward(per_key, mode):
+    """Ragged sequences (a chunk plus a tail, two chunks plus a tail, one
+    short sequence), a random initial state, d_o and d_state_out: every
+    gradient of the chunk-level pass equals the token pass's to rounding,
+    the gradient at the last chunk's end is d_state_out, and the pass's
+    d_state_in is the one it carries out of the first chunk."""
+    rng = np.random.default_rng(95 + 2 * per_key + (mode != "none"))
+    x, cu = _case(rng, [70, 130, 9], 2, 16, 64, per_key)
+    o, s = oracle.recurrence(*x.values(), cu, per_key_gate=per_key, qdq=mode)
+    Wo, Ws = rng.standard_normal(o.shape), rng.standard_normal(s.shape)
+    ref = bw.backward(*x.values(), cu, Wo, Ws, per_key_gate=per_key, qdq=mode)
+    got = bw.chunked_backward(*x.values(), cu, Wo, Ws, per_key_gate=per_key, qdq=mode,
+                              record=True)
+    for name, a, b in zip(["dq", "dk", "dv", "dg", "dbeta", "dstate_in"], ref, got):
+        err = np.abs(a - b).max() / np.abs(a).max()
+        assert err < 1e-12, f"{name}: relative difference {err:.2e}"
+    dH_end = got[6]
+    for s_i, L in enumerate([70, 130, 9]):
+        last = (L - 1) // 64
+        for h in range(2):
+            np.testing.assert_array_equal(dH_end[(s_i, h, last)], Ws[s_i, h])

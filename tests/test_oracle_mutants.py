@@ -120,6 +120,16 @@ BWD_MUTANTS = [
      "per_key_gate=per_key_gate, qdq=\"none\",\n                              boundary_every=boundary_every, record=True)"),
     ("forward misses the partial last chunk", "return (t + 1) % every == 0 or t == L - 1",
      "return (t + 1) % every == 0"),
+    ("chunk: state adjoint without the chunk decay",
+     "+ gamma[n - 1][:, None] * dHn - W.T @ dVn", "+ dHn - W.T @ dVn"),
+    ("chunk: solve adjoint untransposed", "dA = low_strict * (-(T.T @ dT @ T.T))",
+     "dA = low_strict * (-(T @ dT @ T))"),
+    ("chunk: gate gradient not summed back", "dg = np.cumsum(dG[::-1], axis=0)[::-1]",
+     "dg = dG"),
+    ("chunk: end-decay adjoint sign", "dG -= dEK", "dG += dEK"),
+    ("chunk: A_qk adjoint above the diagonal", "dAqk = low * (scale * (dO @ Vn.T))",
+     "dAqk = scale * (dO @ Vn.T)"),
+    ("chunk: dbeta misses the A term", "dbeta += np.sum(dA * KK, axis=1)", "dbeta += 0.0"),
 ]
 
 BWD_PINS = [
@@ -132,6 +142,10 @@ BWD_PINS = [
     ("finite differences (kda)", lambda: bwd.test_backward_matches_finite_differences_qdq_off(True)),
     ("straight through (gdn, fp8)", lambda: bwd.test_backward_is_straight_through(False, "fp8_tile64")),
     ("straight through (kda, int8)", lambda: bwd.test_backward_is_straight_through(True, "int8_g32")),
+    ("chunked = token (gdn, int8)",
+     lambda: bwd.test_chunked_backward_matches_token_backward(False, "int8_g32")),
+    ("chunked = token (kda, none)",
+     lambda: bwd.test_chunked_backward_matches_token_backward(True, "none")),
 ]
 
 # The pins, cheapest first: a case stops at the first one that fails.
