@@ -15,7 +15,8 @@ Modes:
 * :func:`oracle.backward.backward` - the fp64 reverse pass of the token
   recurrence with the state QDQ passed straight through;
   :func:`oracle.backward.chunked_backward` - the same gradients chunk by
-  chunk (the adjoint of the chunked WY form), pinned to the token pass.
+  chunk (the adjoint of the chunked WY form), pinned to the token pass, and
+  :func:`oracle.backward.chunk_state_gradient`, its sequential part alone.
 
 Pins: every function here is checked by ``tests/test_oracle_*.py`` against
 closed forms, invariants, special cases and library routines (see the

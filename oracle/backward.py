@@ -290,3 +290,21 @@ def chunked_backward(q, k, v, g, beta, state_in, cu_seqlens, do, dstate_out, *,
     if record:
         return dq, dk, dv, dg, dbeta, dst, dH_end
     return dq, dk, dv, dg, dbeta, dst
+
+
+def chunk_state_gradient(Q, K, V, g, beta, H0, dO, dHn, *, scale: float):
+    """The sequential part of :func:`chunk_backward_step` alone: the gradient
+    with respect to the chunk-start state,
+    dH0 = diag(gamma_n) dHn - W^T (K * E) dHn + scale ((Q * gamma)^T - W^T A_qk^T) dO,
+    whose bracketed term and W, K * E, A_qk do not depend on dHn."""
+    n, d_k = K.shape
+    G = np.cumsum(g, axis=0)
+    gamma = np.exp(G)
+    D = np.exp(G[:, None, :] - G[None, :, :])
+    E = np.exp(G[n - 1][None, :] - G)
+    A = np.tril(beta[:, None] * np.einsum("rc,ic,ric->ri", K, K, D), k=-1)
+    T = np.linalg.inv(np.eye(n) + A)
+    W = T @ (beta[:, None] * (K * gamma))
+    Aqk = np.tril(np.einsum("rc,ic,ric->ri", Q, K, D))
+    bracket = scale * ((Q * gamma).T @ dO - W.T @ (Aqk.T @ dO))
+    return gamma[n - 1][:, None] * dHn - W.T @ ((K * E) @ dHn) + bracket

@@ -8,7 +8,9 @@
   gradient) match the backward's gradients;
 * closed forms at beta = 0, g = 0 (the state stays H0);
 * the chunk-level reverse pass (the adjoint of the chunked WY form, chunk by
-  chunk from the forward's chunk-start states) equals the token reverse pass.
+  chunk from the forward's chunk-start states) equals the token reverse pass,
+  and its sequential part run alone (the state-gradient chain) gives the same
+  chunk-end state gradients.
 """
 
 import numpy as np
@@ -145,3 +147,32 @@ def test_chunked_backward_matches_token_backward(per_key, mode):
         last = (L - 1) // 64
         for h in range(2):
             np.testing.assert_array_equal(dH_end[(s_i, h, last)], Ws[s_i, h])
+
+
+@pytest.mark.parametrize("per_key", [False, True])
+def test_state_gradient_chain_alone(per_key):
+    """The sequential part of the chunk adjoint run by itself from the end
+    (dH_n of the last chunk = d_state_out) reproduces the chunk-end state
+    gradients the full chunk-level pass records, and d_state_in."""
+    rng = np.random.default_rng(97 + per_key)
+    lengths = [150, 64]
+    x, cu = _case(rng, lengths, 1, 16, 64, per_key)
+    o, s = oracle.recurrence(*x.values(), cu, per_key_gate=per_key, qdq="int8_g32")
+    Wo, Ws = rng.standard_normal(o.shape), rng.standard_normal(s.shape)
+    got = bw.chunked_backward(*x.values(), cu, Wo, Ws, per_key_gate=per_key, qdq="int8_g32",
+                              record=True)
+    dH_end, dst = got[6], got[5]
+    _, _, _, states = bw.forward(*x.values(), cu, per_key_gate=per_key, qdq="int8_g32",
+                                 record=True)
+    scale = 1 / np.sqrt(16)
+    for s_i, L in enumerate(lengths):
+        t0 = int(cu[s_i])
+        dH = Ws[s_i, 0].copy()
+        for ci in range((L - 1) // 64, -1, -1):
+            np.testing.assert_allclose(dH, dH_end[(s_i, 0, ci)], rtol=1e-12, atol=1e-12)
+            a, b = t0 + 64 * ci, t0 + min(64 * ci + 64, L)
+            gc = x["g"][a:b, 0] if per_key else x["g"][a:b, 0][:, None] * np.ones((1, 16))
+            dH = bw.chunk_state_gradient(x["q"][a:b, 0], x["k"][a:b, 0], x["v"][a:b, 0], gc,
+                                         x["beta"][a:b, 0], states[(s_i, 0, 64 * ci)],
+                                         Wo[a:b, 0], dH, scale=scale)
+        np.testing.assert_allclose(dH, dst[s_i, 0], rtol=1e-12, atol=1e-12)
