@@ -14,6 +14,13 @@ workloads fix, each added up from its parts:
   written 131,072 B, q/k/v 768 B, o 256 B, g and beta 8 B: 132,104 B;
   packed INT8 g32: codes 32,768 B, scales 4,096 B, the same 1,032 B of
   token data: 37,896 B;
+* KDA prefill workload (B=2, H=32, T=8192, d=128, bf16, per-key fp32 log
+  gates, zero initial state): q, k, v 402,653,184 B; g 268,435,456 B;
+  beta 2,097,152 B; o 134,217,728 B; states written 4,194,304 B:
+  811,597,824 B per call;
+* packed varlen workload (64 sequences, H=16, d=128, bf16, scalar gate,
+  random initial state read and written): 1,032 B per head-token plus
+  134,217,728 B of state;
 * backward on the GDN workload: 679,477,248 B (inputs read once, fp32
   gradients written once);
 * the recorded DRAM traffic is reported only for the sources it was taken
@@ -33,6 +40,27 @@ def test_prefill_bytes_gdn_workload():
     assert bench.prefill_bytes(4 * 4096, 4, 16, 128, 128, 2, True, False) == got + 4_194_304
     assert (bench.prefill_bytes(4 * 4096, 4, 16, 128, 128, 2, False, True)
             == got + tok * 127 * 4)
+
+
+def test_prefill_bytes_kda_workload():
+    tok = 2 * 8192 * 32
+    parts = tok * 3 * 128 * 2 + tok * 128 * 4 + tok * 4 + tok * 128 * 2 + 2 * 32 * 128 * 128 * 4
+    total = 402_653_184 + 268_435_456 + 2_097_152 + 134_217_728 + 4_194_304
+    assert parts == total == 811_597_824
+    got = bench.prefill_bytes(2 * 8192, 2, 32, 128, 128, 2, state_in=False, per_key=True)
+    assert got == 811_597_824
+
+
+def test_prefill_bytes_varlen_workload():
+    import gdn_synth as gs
+    lengths = gs.generate(gs.small_case("varlen", decode_steps=0))["lengths"]
+    tokens = sum(lengths)
+    head_tokens = tokens * 16
+    per_head_token = 3 * 128 * 2 + 128 * 2 + 4 + 4  # q, k, v, o, g, beta
+    state = 64 * 16 * 128 * 128 * 4 * 2            # read and written
+    assert per_head_token == 1032 and state == 134_217_728
+    got = bench.prefill_bytes(tokens, 64, 16, 128, 128, 2, state_in=True, per_key=False)
+    assert got == head_tokens * per_head_token + state
 
 
 def test_backward_bytes_gdn_workload():
